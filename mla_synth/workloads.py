@@ -1,0 +1,309 @@
+"""Named MLA decode workloads and their seeded generator.
+
+Shapes follow the DeepSeek-V2/V3 dimensions the pages quote for the latent
+cache (kv_lora_rank 512 + rope dim 64 = 576 values per token per layer:
+"GQA, MQA ve MLA", section "Multi-head latent attention (MLA)"), plus a tiny
+fp32 shape that the fp64 oracle finishes in milliseconds.
+
+Draw order for one workload, all from one CPU ``torch.Generator`` seeded
+with ``workload.seed`` (fixed so that every consumer sees identical values):
+
+1. weights, in the order W_DKV, W_KR, (W_DQ, W_UQ) or W_Q, W_UK, W_UV, W_O;
+   each ``randn(fan_in, fan_out) * fan_in ** -0.5`` in fp32, then rounded to
+   the workload dtype (round-to-nearest-even for bf16);
+2. the cached context lengths (``randint(lo, hi + 1, (batch,))`` when ragged);
+3. the new tokens' hidden states ``x_new`` ``[batch * n_q, hidden]``, N(0, 1);
+4. the cached rows: either hidden states ``x_cached`` ``[L, hidden]`` whose
+   latent rows the append step produces (tiny shape), or latent rows
+   ``[sum L_b, d_c + d_r]`` drawn N(0, 1) directly, optionally with a
+   Bernoulli(frac) subset of rows scaled by ``spike_scale``;
+5. the physical block permutation of the paged pool (``randperm``), when
+   the workload asks for shuffled blocks.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from dataclasses import dataclass, field
+from typing import Dict, Optional, Sequence, Tuple
+
+import torch
+
+
+@dataclass(frozen=True)
+class MLAShape:
+    """Per-layer MLA dimensions (row-vector convention, weights ``[in, out]``)."""
+
+    name: str
+    hidden: int
+    n_heads: int
+    d_c: int          # joint KV latent width (kv_lora_rank)
+    d_r: int          # decoupled RoPE key width, shared by all heads
+    qk_nope: int      # per-head no-position query/key width
+    v_head: int       # per-head value width
+    q_lora: int       # 0: queries are projected directly by W_Q
+    rope_theta: float = 10000.0
+    dtype: str = "bf16"  # "bf16" or "f32": storage type of weights, cache and activations
+    block_size: int = 64
+
+    @property
+    def row(self) -> int:
+        return self.d_c + self.d_r
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+    @property
+    def elem_bytes(self) -> int:
+        return 2 if self.dtype == "bf16" else 4
+
+    def weight_shapes(self) -> Dict[str, Tuple[int, int]]:
+        """Weight name -> (fan_in, fan_out), in draw order."""
+        H = self.n_heads
+        q_width = H * (self.qk_nope + self.d_r)
+        shapes = {
+            "W_DKV": (self.hidden, self.d_c),
+            "W_KR": (self.hidden, self.d_r),
+        }
+        if self.q_lora > 0:
+            shapes["W_DQ"] = (self.hidden, self.q_lora)
+            shapes["W_UQ"] = (self.q_lora, q_width)
+        else:
+            shapes["W_Q"] = (self.hidden, q_width)
+        # W_UK and W_UV map the latent (fan_in d_c) to per-head key / value.
+        shapes["W_UK"] = (self.d_c, H * self.qk_nope)
+        shapes["W_UV"] = (self.d_c, H * self.v_head)
+        shapes["W_O"] = (H * self.v_head, self.hidden)
+        return shapes
+
+
+SHAPES: Dict[str, MLAShape] = {
+    "tiny": MLAShape("tiny", hidden=256, n_heads=4, d_c=64, d_r=16, qk_nope=32,
+                     v_head=32, q_lora=0, dtype="f32"),
+    "v2": MLAShape("v2", hidden=5120, n_heads=128, d_c=512, d_r=64, qk_nope=128,
+                   v_head=128, q_lora=1536, dtype="bf16"),
+    "v3": MLAShape("v3", hidden=7168, n_heads=128, d_c=512, d_r=64, qk_nope=128,
+                   v_head=128, q_lora=1536, dtype="bf16"),
+}
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One decode step over a batch of sequences.
+
+    ``lengths`` fixes the cached context length of every sequence; when it is
+    ``None`` the lengths are drawn uniformly from ``[len_lo, len_hi]``.  Each
+    sequence then appends ``n_q`` new latent rows (positions ``L_b .. L_b +
+    n_q - 1``) and each new token attends causally, itself included.
+    """
+
+    name: str
+    shape: MLAShape
+    batch: int
+    n_q: int = 1
+    lengths: Optional[Tuple[int, ...]] = None
+    len_lo: int = 0
+    len_hi: int = 0
+    cached_from_append: bool = False   # cached rows come from x_cached via the append step
+    shuffled_blocks: bool = False
+    spike_frac: float = 0.0
+    spike_scale: float = 1.0
+    seed: int = 0
+    description: str = ""
+
+    @property
+    def n_tok(self) -> int:
+        return self.batch * self.n_q
+
+
+WORKLOADS: Dict[str, Workload] = {
+    "tiny_f32_b1_l128": Workload(
+        "tiny_f32_b1_l128", SHAPES["tiny"], batch=1, n_q=1, lengths=(128,),
+        cached_from_append=True,
+        description="tiny fp32 MLA, 1 layer, 128 cached tokens + 1 decode token"),
+    "v2_b16_l4096": Workload(
+        "v2_b16_l4096", SHAPES["v2"], batch=16, n_q=1, lengths=(4096,) * 16,
+        description="DeepSeek-V2-shaped decode, batch 16 x 4096 cached tokens, 1 new token each"),
+    "v3_b64_ragged1k_8k": Workload(
+        "v3_b64_ragged1k_8k", SHAPES["v3"], batch=64, n_q=1, len_lo=1024, len_hi=8192,
+        shuffled_blocks=True,
+        description="DeepSeek-V3-shaped decode, batch 64, ragged lengths U[1024, 8192], "
+                    "64-token pages in shuffled order"),
+    "v3_b4_long": Workload(
+        "v3_b4_long", SHAPES["v3"], batch=4, n_q=1, lengths=(65536, 131072, 32768, 100000),
+        spike_frac=0.01, spike_scale=8.0,
+        description="V3-shaped long-context split-KV stress, contexts 65536/131072/32768/100000, "
+                    "1% of latent rows scaled x8"),
+    "v3_b128_nq2_ragged512_16k": Workload(
+        "v3_b128_nq2_ragged512_16k", SHAPES["v3"], batch=128, n_q=2, len_lo=512, len_hi=16384,
+        description="V3-shaped multi-token decode, batch 128, 2 causal query tokens per sequence, "
+                    "ragged lengths U[512, 16384], append 2 rows then attend"),
+}
+
+
+def reduced(wl: Workload, *, batch: Optional[int] = None,
+            lengths: Optional[Sequence[int]] = None,
+            len_lo: Optional[int] = None, len_hi: Optional[int] = None,
+            n_q: Optional[int] = None, seed: Optional[int] = None,
+            name: Optional[str] = None) -> Workload:
+    """The same shape and structure at a smaller batch / context size."""
+    kw = {}
+    if lengths is not None:
+        kw["lengths"] = tuple(int(v) for v in lengths)
+        kw["batch"] = len(kw["lengths"])
+    if batch is not None:
+        kw["batch"] = batch
+        if lengths is None and wl.lengths is not None:
+            base = wl.lengths
+            kw["lengths"] = tuple(base[i % len(base)] for i in range(batch))
+    if len_lo is not None:
+        kw["len_lo"] = len_lo
+    if len_hi is not None:
+        kw["len_hi"] = len_hi
+    if n_q is not None:
+        kw["n_q"] = n_q
+    if seed is not None:
+        kw["seed"] = seed
+    kw["name"] = name or (wl.name + "_reduced")
+    return dataclasses.replace(wl, **kw)
+
+
+@dataclass
+class WorkloadData:
+    """Seeded inputs of one workload, as CPU tensors in the workload dtype."""
+
+    workload: Workload
+    weights: Dict[str, torch.Tensor]
+    cached_len: torch.Tensor              # int64 [B]: rows already in the cache
+    x_new: torch.Tensor                   # [B*n_q, hidden], row b*n_q + j is token j of seq b
+    cached_rows: Optional[torch.Tensor]   # [sum L_b, d_c + d_r] latent rows (None if from append)
+    x_cached: Optional[torch.Tensor]      # [sum L_b, hidden] (only when cached_from_append)
+    spike_mask: Optional[torch.Tensor]    # bool [sum L_b] rows scaled by spike_scale
+    block_table: torch.Tensor             # int32 [B, max_blocks]
+    num_blocks: int
+    row_offsets: torch.Tensor = field(default=None)  # int64 [B+1] start of seq b in cached rows
+
+    @property
+    def seq_lens(self) -> torch.Tensor:
+        """Rows per sequence after the append step (cached + new)."""
+        return self.cached_len + self.workload.n_q
+
+    def new_positions(self) -> torch.Tensor:
+        """int32 [B*n_q]: absolute position of each new token (0-based)."""
+        n_q = self.workload.n_q
+        j = torch.arange(n_q, dtype=torch.int64)
+        return (self.cached_len[:, None] + j[None, :]).reshape(-1).to(torch.int32)
+
+    def new_seq_idx(self) -> torch.Tensor:
+        """int32 [B*n_q]: sequence index of each new token."""
+        n_q = self.workload.n_q
+        return torch.arange(self.workload.batch, dtype=torch.int32).repeat_interleave(n_q)
+
+    def seq_rows(self, b: int) -> torch.Tensor:
+        """Cached latent rows of sequence b (before the append step)."""
+        s, e = int(self.row_offsets[b]), int(self.row_offsets[b + 1])
+        return self.cached_rows[s:e]
+
+
+def _draw_weights(shape: MLAShape, g: torch.Generator) -> Dict[str, torch.Tensor]:
+    out = {}
+    for name, (fan_in, fan_out) in shape.weight_shapes().items():
+        w = torch.randn(fan_in, fan_out, generator=g, dtype=torch.float32)
+        w.mul_(fan_in ** -0.5)
+        out[name] = w.to(shape.torch_dtype)
+    return out
+
+
+def _draw_rows(n: int, width: int, dtype: torch.dtype, g: torch.Generator,
+               chunk: int = 1 << 20) -> torch.Tensor:
+    """N(0, 1) rows drawn in row chunks (bounded fp32 temporaries)."""
+    out = torch.empty(n, width, dtype=dtype)
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        out[s:e] = torch.randn(e - s, width, generator=g, dtype=torch.float32).to(dtype)
+    return out
+
+
+def generate(wl: Workload, *, with_weights: bool = True) -> WorkloadData:
+    """Draw every input of ``wl`` from its seed (see the module docstring)."""
+    shape = wl.shape
+    g = torch.Generator().manual_seed(wl.seed)
+    dt = shape.torch_dtype
+
+    weights: Dict[str, torch.Tensor] = {}
+    if with_weights:
+        weights = _draw_weights(shape, g)
+    else:
+        # Keep the stream aligned with the with-weights draw order.
+        for _name, (fan_in, fan_out) in shape.weight_shapes().items():
+            torch.randn(fan_in, fan_out, generator=g, dtype=torch.float32)
+
+    if wl.lengths is not None:
+        if len(wl.lengths) != wl.batch:
+            raise ValueError("lengths must have one entry per sequence")
+        cached_len = torch.tensor(wl.lengths, dtype=torch.int64)
+    else:
+        cached_len = torch.randint(wl.len_lo, wl.len_hi + 1, (wl.batch,), generator=g,
+                                   dtype=torch.int64)
+
+    x_new = torch.randn(wl.n_tok, shape.hidden, generator=g, dtype=torch.float32).to(dt)
+
+    total = int(cached_len.sum())
+    row_offsets = torch.zeros(wl.batch + 1, dtype=torch.int64)
+    row_offsets[1:] = torch.cumsum(cached_len, 0)
+    cached_rows = x_cached = spike_mask = None
+    if wl.cached_from_append:
+        x_cached = torch.randn(total, shape.hidden, generator=g, dtype=torch.float32).to(dt)
+    else:
+        cached_rows = _draw_rows(total, shape.row, dt, g)
+        if wl.spike_frac > 0.0:
+            spike_mask = torch.rand(total, generator=g) < wl.spike_frac
+            idx = spike_mask.nonzero().squeeze(1)
+            cached_rows[idx] = (cached_rows[idx].to(torch.float32) * wl.spike_scale).to(dt)
+
+    bs = shape.block_size
+    blocks_per_seq = (cached_len + wl.n_q + bs - 1) // bs
+    num_blocks = int(blocks_per_seq.sum())
+    max_blocks = int(blocks_per_seq.max()) if wl.batch > 0 else 1
+    logical = torch.arange(num_blocks, dtype=torch.int64)
+    if wl.shuffled_blocks:
+        physical = torch.randperm(num_blocks, generator=g)
+    else:
+        physical = logical
+    block_table = torch.full((wl.batch, max(max_blocks, 1)), -1, dtype=torch.int32)
+    start = 0
+    for b in range(wl.batch):
+        nb = int(blocks_per_seq[b])
+        block_table[b, :nb] = physical[start:start + nb].to(torch.int32)
+        start += nb
+
+    return WorkloadData(wl, weights, cached_len, x_new, cached_rows, x_cached, spike_mask,
+                        block_table, num_blocks, row_offsets)
+
+
+def build_pool(data: WorkloadData, rows: Optional[torch.Tensor] = None,
+               fill: float = float("nan")) -> torch.Tensor:
+    """Scatter cached latent rows into a paged pool ``[num_blocks, block, d_c + d_r]``.
+
+    Pure data movement: row ``t`` of sequence ``b`` goes to
+    ``pool[block_table[b, t // block], t % block]``.  Slots no sequence has
+    written yet keep ``fill`` (NaN by default), so a consumer that reads past
+    a sequence's valid rows is caught.
+    """
+    wl = data.workload
+    shape = wl.shape
+    bs = shape.block_size
+    src = data.cached_rows if rows is None else rows
+    pool = torch.full((max(data.num_blocks, 1), bs, shape.row), fill, dtype=shape.torch_dtype)
+    flat = pool.view(-1, shape.row)
+    for b in range(wl.batch):
+        L = int(data.cached_len[b])
+        if L == 0:
+            continue
+        t = torch.arange(L, dtype=torch.int64)
+        phys = data.block_table[b].to(torch.int64)[t // bs]
+        dst = phys * bs + (t % bs)
+        s = int(data.row_offsets[b])
+        flat[dst] = src[s:s + L]
+    return pool
