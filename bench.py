@@ -1,0 +1,385 @@
+"""Benchmark of the MLA latent-KV decode step on B200 (one JSON line on rank 0).
+
+A step is one pass of the whole decode path over one batch: latent append,
+absorbed queries, split-KV decode, split combine, output projection.  The
+default workload is the DeepSeek-V3-shaped decode (batch 64, ragged cached
+lengths U[1024, 8192] + 1 new token each, 64-token pages in shuffled order,
+seed 0): the configuration on which the decode roofline target is stated.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 oracle on the host cores
+
+Timing: every step is bracketed by CUDA events on the stream the library
+launches on; the L2 is flushed (a 256 MiB write) before every step, outside
+the events; K steps run between a barrier + synchronize on both sides; with
+N > 1 processes (torchrun), each rank runs its own replica of the workload
+(weak scaling, no collective on the data path) and the step time is the max
+over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+import torch
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+from mla_synth import WORKLOADS, device_inputs, generate  # noqa: E402
+
+DEFAULT_WORKLOAD = "v3_b64_ragged1k_8k"
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------- helpers
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), \
+        int(os.environ.get("LOCAL_RANK", 0))
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank's replica draws its own inputs (weak scaling)."""
+    return base_seed + rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, device=None) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def measured_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted((ROOT / "mla_latent_kv_39_b200" / "csrc").glob("*")):
+        h.update(p.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if the
+    kernel sources are unchanged since it was taken (else None)."""
+    p = ROOT / "profiles" / "decode_traffic.json"
+    if not p.exists():
+        return None
+    d = json.loads(p.read_text())
+    if d.get("source_hash") != kernel_source_hash() or d.get("workload") != workload:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.rows, self.proc = index, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [s.strip() for s in line.split(",")]
+            if len(parts) == 6:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[2 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_sample(wl, budget_s: float = 15.0, max_seqs: int = 64, data=None, W=None, first: int = 0):
+    """Time the fp64 oracle (decompressed order) on whole sequences of ``wl``
+    until ``budget_s`` of CPU time is spent; returns (tokens/s, sample text, cores)."""
+    import numpy as np
+    import oracle
+    data = data if data is not None else generate(wl)
+    shape = wl.shape
+    W = W if W is not None else {k: oracle.to64(v) for k, v in data.weights.items()}
+    done_tok, t_spent, seqs = 0, 0.0, 0
+    for i in range(min(wl.batch, max_seqs)):
+        b = (first + i) % wl.batch
+        s, e = int(data.row_offsets[b]), int(data.row_offsets[b + 1])
+        rows = oracle.to64(data.cached_rows[s:e]) if data.cached_rows is not None else None
+        toks = slice(b * wl.n_q, (b + 1) * wl.n_q)
+        t0 = time.perf_counter()
+        if rows is None:
+            c, kr = oracle.latent_rows(data.x_cached[s:e], W["W_DKV"], W["W_KR"], np.arange(e - s),
+                                       shape.rope_theta, shape.dtype)
+        else:
+            c, kr = rows[:, :shape.d_c], rows[:, shape.d_c:]
+        pos = data.new_positions().numpy()[toks]
+        oracle.decode_step(shape, W, oracle.to64(data.x_new[toks]), pos, [c], [kr], wl.n_q,
+                           order="decompressed")
+        t_spent += time.perf_counter() - t0
+        done_tok += wl.n_q
+        seqs += 1
+        if t_spent >= budget_s:
+            break
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    threads = torch.get_num_threads()
+    sample = (f"{seqs} of {wl.batch} sequences ({done_tok} query tokens, full decode step: append, "
+              f"queries, decompressed attention over all heads, output projection) in {t_spent:.1f} s")
+    return done_tok / t_spent, sample, min(cores, max(threads, 1))
+
+
+# ----------------------------------------------------------------- main arms
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    wl = WORKLOADS[args.workload]
+    data = generate(wl)
+    W = {k: oracle.to64(v) for k, v in data.weights.items()}
+    per_step = []
+    sample = ""
+    cores = 1
+    n = args.steps + args.warmup
+    step_budget = max(30.0, min(180.0, 6.0 * n)) / n
+    for i in range(n):
+        tps, sample, cores = oracle_sample(wl, budget_s=step_budget, max_seqs=wl.batch, data=data, W=W,
+                                           first=i)
+        if i >= args.warmup:
+            per_step.append(tps)
+    value = statistics.mean(per_step)
+    line = {
+        "impl": "reference",
+        "metric": "MLA decode tokens/s (fp64 CPU oracle, decompressed order)",
+        "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * wl.n_tok / value if value else None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": wl.name, "batch": wl.batch, "n_q": wl.n_q},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    import mla_latent_kv_39_b200 as mla
+
+    base = WORKLOADS[args.workload]
+    import dataclasses
+    wl = dataclasses.replace(base, seed=rank_seed(base.seed, rank))
+    data = generate(wl)
+    dev = device_inputs(data, device)
+    cfg = mla.Config.from_shape(wl.shape)
+    cache = mla.Cache(dev["pool"], dev["block_table"])
+    layer = mla.DecodeLayer(cfg, dev["weights"], cache, wl.batch, wl.n_q, args.max_workers)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    x, seq_idx, pos, seq_lens = dev["x_new"], dev["seq_idx"], dev["pos"], dev["seq_lens"]
+    # every step appends the same positions again (the appended rows are rewritten identically)
+
+    def one_step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        layer.append(x, seq_idx, pos)
+        layer.queries(x, pos)
+        if ev is not None:
+            ev[1].record(stream)
+        layer.decode(seq_lens)
+        if ev is not None:
+            ev[2].record(stream)
+        layer.combine()
+        layer.project()
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        one_step()
+    torch.cuda.synchronize()
+    mla.check_device_error()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    launches0 = mla.mla_kernel_launches()
+    barrier()
+    wall0 = time.perf_counter()
+    with ClockSampler(local) as clocks:
+        for k in range(args.steps):
+            flush.fill_(1)
+            one_step(events[k])
+        barrier()
+    wall = time.perf_counter() - wall0
+    launches = mla.mla_kernel_launches() - launches0
+    mla.check_device_error()
+    step_ms = [e[0].elapsed_time(e[3]) for e in events]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in events]
+    total_ms = max_over_ranks(sum(step_ms), device)
+    tokens = sum_over_ranks(float(wl.n_tok * args.steps), device)
+    value = tokens / (total_ms / 1000.0)
+
+    # end to end through the public API with host (pinned) buffers
+    x_h = data.x_new.pin_memory()
+    seq_idx_h = data.new_seq_idx().pin_memory()
+    pos_h = data.new_positions().pin_memory()
+    seq_lens_h = data.seq_lens.to(torch.int32).pin_memory()
+    y_h = torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (x_h, seq_idx_h, pos_h, seq_lens_h))
+    d2h = y_h.numel() * y_h.element_size()
+    for _ in range(max(1, args.warmup)):
+        flush.fill_(1)
+        layer.step_from_host(x_h, seq_idx_h, pos_h, seq_lens_h, y_h, stream)
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier()
+    for k in range(args.steps):
+        flush.fill_(1)
+        e2e_ev[k][0].record(stream)
+        layer.step_from_host(x_h, seq_idx_h, pos_h, seq_lens_h, y_h, stream)
+        e2e_ev[k][1].record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev), device)
+    e2e_value = tokens / (e2e_ms / 1000.0)
+
+    peaks = measured_peaks()
+    cache_bytes = int(data.seq_lens.sum()) * wl.shape.row * wl.shape.elem_bytes
+    dec_avg_s = statistics.mean(dec_ms) / 1000.0
+    achieved = cache_bytes / dec_avg_s / 1e9
+    traffic = recorded_traffic(wl.name)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        tps, sample, cores = oracle_sample(wl, budget_s=args.cpu_budget, max_seqs=wl.batch)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+    ms_per_step = total_ms / args.steps
+    line = {
+        "metric": "MLA decode tokens/s and latent-KV GB/s (% of HBM roofline), 1 B200",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.shape.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded; random-init weights of the V3 layer shape)",
+        "config": {"workload": wl.name, "batch": wl.batch, "n_q": wl.n_q,
+                   "cached_len": (f"{int(data.cached_len.min())}..{int(data.cached_len.max())}"),
+                   "cache_rows": int(data.seq_lens.sum()), "block_size": wl.shape.block_size,
+                   "page_order": "shuffled" if wl.shuffled_blocks else "in order",
+                   "l2": "flushed (256 MiB write) before every step, outside the timed events",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "latent_kv_gbs": achieved,
+        "decode_ms": statistics.mean(dec_ms),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "kernel": "mla_decode call (plan + decode kernels)",
+                     "algorithmic_bytes_per_launch": cache_bytes,
+                     "peak_source": peaks["source"]},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": wall,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--max-workers", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+def main(argv=None):
+    args = parse(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

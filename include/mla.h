@@ -1,0 +1,210 @@
+/*
+ * mla.h - C ABI of the MLA latent-KV decode library (libmla.so).
+ *
+ * Multi-head Latent Attention caches, per token and layer, one compressed
+ * latent c_KV (d_c values) plus one small decoupled rotary key k_R (d_r
+ * values, shared by all heads) instead of per-head K and V.  At decode time
+ * the key/value up-projections are folded into the query and output sides
+ * (matrix absorption), so per-head K and V are never materialised.
+ *
+ * Sources (by page title and section):
+ *  [P2] "Multi-head Latent Attention (MLA) Nedir?" (yapayzekasozluk.tr),
+ *       section "MLA nasıl çalışır?" (Compression, Decompression, Decoupled
+ *       RoPE, query compression) and "MLA ve diğer optimizasyonlarla
+ *       ilişkisi" (page-based caches hold the smaller latent vectors).
+ *  [P4] "GQA, MQA ve MLA: attention KV cache'i nasıl belirler" (LLMScale),
+ *       section "Multi-head latent attention (MLA)" (what one cache row holds).
+ *  [P5] "MLA · latent KV, decoupled RoPE và matrix absorption" (openarchlab),
+ *       section 1 "Định nghĩa" (absorption into the query and output
+ *       matrices; RoPE kept on a separate branch), section 2 "Luồng" (project
+ *       hidden to latent -> write the cache -> read and project the output).
+ *
+ * Conventions shared by every entry point
+ *  - Row-vector convention y = x W.  Every weight is stored [in, out],
+ *    row-major, in the config's storage dtype (bf16 or f32).
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *    except where an argument says otherwise.  `stream` is a cudaStream_t
+ *    (NULL = legacy default stream).  Every call is asynchronous on `stream`
+ *    and never synchronises, except mla_get_device_error.
+ *  - Ownership: the caller owns every buffer, including the workspaces whose
+ *    sizes the *_workspace_size queries return.  The library allocates no
+ *    device memory.  Its only device state is one error word per device
+ *    (a file-scope __device__ variable).
+ *  - Synchronous errors (null pointers, unsupported dimensions, workspace too
+ *    small, a failed launch) return a negative mla_status before or at launch
+ *    and leave outputs untouched.  Data-dependent errors found on the device
+ *    (a block id outside the pool, a position past a sequence's block table,
+ *    a sequence shorter than its query count) skip the offending work,
+ *    record the first such error in the device error word, and surface
+ *    through mla_get_device_error.  No C++ exception crosses this ABI.
+ *  - Storage dtype: MLA_BF16 (bf16 storage, fp32 accumulation) or MLA_F32
+ *    (fp32 storage and arithmetic on CUDA cores, for small shapes).
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_ABI_VERSION 1
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = -1,  /* null pointer, negative size, inconsistent config */
+  MLA_ERR_UNSUPPORTED = -2,  /* dimensions this build has no kernel for */
+  MLA_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed */
+  MLA_ERR_BOUNDS = -4,       /* (device) block id / position / length out of range */
+  MLA_ERR_TIMEOUT = -5,      /* (device) a bounded wait gave up */
+  MLA_ERR_WORKSPACE = -6     /* workspace too small, or not written by mla_decode */
+} mla_status;
+
+typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype;
+
+/* Per-layer MLA dimensions. */
+typedef struct {
+  int32_t hidden;        /* model width */
+  int32_t n_heads;       /* H */
+  int32_t d_c;           /* latent width (kv_lora_rank) */
+  int32_t d_r;           /* decoupled RoPE key width (even), one key shared by all heads */
+  int32_t qk_nope;       /* per-head no-position query/key width */
+  int32_t v_head;        /* per-head value width */
+  int32_t q_lora;        /* query latent width; 0 = no query compression (W_Q used directly) */
+  double rope_theta;     /* RoPE base; pair (2i, 2i+1) turns by pos * theta^(-2i/d_r) */
+  float softmax_scale;   /* 0 -> 1/sqrt(qk_nope + d_r) */
+  int32_t block_size;    /* tokens per cache page */
+  int32_t dtype;         /* mla_dtype */
+} mla_config;
+
+/* Paged latent cache of one layer ([P2] "MLA ve diğer optimizasyonlarla ilişkisi").
+ * pool:        [num_blocks, block_size, d_c + d_r] storage dtype; row = [c_KV | k_R].
+ * block_table: int32 [batch, max_blocks_per_seq]; entry (b, k) is the pool block
+ *              holding positions [k*block_size, (k+1)*block_size) of sequence b.
+ * The library reads and writes the pool in place; the caller owns all of it. */
+typedef struct {
+  void* pool;
+  int32_t num_blocks;
+  const int32_t* block_table;
+  int32_t batch;
+  int32_t max_blocks_per_seq;
+} mla_cache;
+
+/* ---------------------------------------------------------------------------
+ * Step 1 - latent append ([P5] section 2 "Luồng", steps 1-2; [P2] Compression
+ * and Decoupled RoPE; [P4] one row = d_c latent values + d_r rotary values).
+ * For each new token t:  c = x_t W_DKV,  k_R = RoPE(x_t W_KR, pos[t]),
+ * and the row [c | k_R], rounded once to the storage dtype, is stored at
+ * pool[block_table[seq_idx[t]][pos[t] / block_size]][pos[t] % block_size].
+ * The bf16 path reproduces the exactly rounded value of the real-number dot
+ * product (fp64 accumulation), so the cache is bit-identical to x W rounded
+ * once to bf16.
+ *   x        [n_tok, hidden]        storage dtype
+ *   W_DKV    [hidden, d_c], W_KR [hidden, d_r]
+ *   seq_idx  int32 [n_tok]   sequence of each token (row of block_table)
+ *   pos      int32 [n_tok]   0-based absolute position of each token
+ *   workspace >= mla_cache_append_workspace_size(cfg, n_tok) bytes
+ * Device errors: a block id outside [0, num_blocks) or a page index outside
+ * [0, max_blocks_per_seq) -> MLA_ERR_BOUNDS, row not written.
+ * ------------------------------------------------------------------------- */
+size_t mla_cache_append_workspace_size(const mla_config* cfg, int32_t n_tok);
+mla_status mla_cache_append(const mla_config* cfg, const void* x, int32_t n_tok,
+                            const void* W_DKV, const void* W_KR,
+                            const int32_t* seq_idx, const int32_t* pos,
+                            const mla_cache* cache, void* workspace, size_t ws_bytes,
+                            void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Step 2 - queries with W_UK absorbed ([P2] query compression; [P5] section 1
+ * "Định nghĩa": the decompression matrix is folded into the query matrix, the
+ * RoPE part stays separate).
+ *   c_Q = x W_DQ (q_lora > 0) ;  q = c_Q W_UQ   (q_lora == 0: q = x W_Q, pass W_Q as W_UQ, W_DQ = NULL)
+ *   head h owns q columns [h(qk_nope+d_r), (h+1)(qk_nope+d_r)): qk_nope no-position
+ *   values then d_r rotary values;  q_rope_h = RoPE(q_R_h, pos[t]);
+ *   q_lat_h = q_nope_h W_UK_h^T  with  W_UK_h = W_UK[:, h qk_nope : (h+1) qk_nope].
+ *   x      [n_tok, hidden];  W_DQ [hidden, q_lora];  W_UQ [q_lora or hidden, H (qk_nope + d_r)]
+ *   W_UK   [d_c, H qk_nope];  pos int32 [n_tok]
+ *   q_lat  [n_tok, H, d_c] (out, storage dtype);  q_rope [n_tok, H, d_r] (out)
+ *   workspace >= mla_absorb_q_workspace_size(cfg, n_tok) bytes
+ * ------------------------------------------------------------------------- */
+size_t mla_absorb_q_workspace_size(const mla_config* cfg, int32_t n_tok);
+mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok,
+                        const void* W_DQ, const void* W_UQ, const void* W_UK,
+                        const int32_t* pos, void* q_lat, void* q_rope,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Step 3 - split-KV decode in latent space ([P5] section 2 "Luồng" step 3:
+ * scores and output from the merged matrices or an equivalent kernel; [P2]
+ * "MLA'nın avantajları ve hesap maliyeti": recompute from the small latent
+ * instead of storing K/V).  For sequence b, query j (token t = b n_q + j,
+ * position p = seq_lens[b] - n_q + j) and head h:
+ *   s_u = (q_lat[t,h] . c_u + q_rope[t,h] . kR_u) * scale   for rows u <= p
+ *   o_lat[t,h] = sum_u softmax(s)_u c_u
+ * The rows of every sequence are split into contiguous page ranges, one per
+ * scheduled worker; each range writes an unnormalised-free partial
+ * (softmax-normalised over its rows) and its log2-sum-exp into `workspace`;
+ * mla_combine merges them.
+ *   q_lat [batch n_q, H, d_c], q_rope [batch n_q, H, d_r]: from mla_absorb_q
+ *   seq_lens int32 [batch]: rows of each sequence INCLUDING the n_q new rows
+ *            (already appended); must satisfy n_q <= seq_lens[b] <=
+ *            max_blocks_per_seq * block_size.
+ *   max_workers: upper bound on parallel workers (0 = sized to the device).
+ *   workspace >= mla_decode_workspace_size(cfg, batch, n_q, max_workers)
+ * Device errors: bad lengths or block ids -> MLA_ERR_BOUNDS (that sequence's
+ * output is zero).
+ * ------------------------------------------------------------------------- */
+size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t n_q,
+                                 int32_t max_workers);
+mla_status mla_decode(const mla_config* cfg, const void* q_lat, const void* q_rope,
+                      int32_t batch, int32_t n_q, const mla_cache* cache,
+                      const int32_t* seq_lens, int32_t max_workers,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Step 4a - split combine (not on the pages; the standard log-sum-exp merge):
+ *   o_lat[t,h] = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),  M = max_s lse_s
+ * over the partials that mla_decode left in `workspace` (same batch, n_q).
+ *   o_lat  float32 [batch n_q, H, d_c] (out)
+ * Returns MLA_ERR_WORKSPACE on the device error word if the workspace was not
+ * written by a matching mla_decode call.
+ * ------------------------------------------------------------------------- */
+mla_status mla_combine(const mla_config* cfg, const void* workspace, size_t ws_bytes,
+                       int32_t batch, int32_t n_q, float* o_lat, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Step 4b - output side with W_UV absorbed ([P5] section 1 "Định nghĩa":
+ * the decompression matrix folded into the output matrix).
+ *   o_h = o_lat_h W_UV_h  (W_UV_h = W_UV[:, h v_head : (h+1) v_head]),
+ *   y   = concat_h(o_h) W_O
+ *   o_lat float32 [n_tok, H, d_c];  W_UV [d_c, H v_head];  W_O [H v_head, hidden]
+ *   y     [n_tok, hidden] storage dtype (out)
+ *   workspace >= mla_out_proj_workspace_size(cfg, n_tok) bytes
+ * ------------------------------------------------------------------------- */
+size_t mla_out_proj_workspace_size(const mla_config* cfg, int32_t n_tok);
+mla_status mla_out_proj(const mla_config* cfg, const float* o_lat, int32_t n_tok,
+                        const void* W_UV, const void* W_O, void* y,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Errors and introspection
+ * ------------------------------------------------------------------------- */
+/* Synchronises `stream`, returns the first device-side error recorded on the
+ * current device since the last call (MLA_OK if none) and clears it.
+ * detail (may be NULL) receives 3 ints describing the failing item. */
+mla_status mla_get_device_error(void* stream, int32_t* detail);
+/* Static description of a status code. */
+const char* mla_status_string(mla_status status);
+/* MLA_ABI_VERSION of the loaded library. */
+int32_t mla_abi_version(void);
+/* Number of CUDA kernels this library has launched in this process, on all
+ * devices (a host-side counter; it never synchronises). */
+int64_t mla_kernel_launches(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* MLA_H_ */

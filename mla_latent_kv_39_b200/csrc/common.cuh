@@ -1,0 +1,87 @@
+// Shared device helpers: the device error word, storage-type conversion,
+// warp reductions, and small host helpers used by every entry point.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "mla.h"
+
+namespace mla {
+
+using bf16 = __nv_bfloat16;
+
+// First device-side error since the last mla_get_device_error: [code, a, b, c].
+// One copy per device that loads the library; kernels only ever set it once
+// (compare-and-swap from zero), so a later error never hides the first one.
+__device__ int g_err[4];
+
+__device__ __forceinline__ void report(int code, int a, int b, int c) {
+  if (atomicCAS(&g_err[0], 0, code) == 0) {
+    g_err[1] = a;
+    g_err[2] = b;
+    g_err[3] = c;
+  }
+}
+
+// ------------------------------------------------------------ storage types
+template <typename T> struct Store;
+
+template <> struct Store<float> {
+  static __device__ __forceinline__ float ld(const float* p) { return *p; }
+  static __device__ __forceinline__ float cvt(float v) { return v; }
+  static __device__ __forceinline__ void st(float* p, float v) { *p = v; }
+  // round a double once to the storage type (nearest, ties to even)
+  static __device__ __forceinline__ void st64(float* p, double v) { *p = __double2float_rn(v); }
+};
+
+template <> struct Store<bf16> {
+  static __device__ __forceinline__ float ld(const bf16* p) { return __bfloat162float(*p); }
+  static __device__ __forceinline__ float cvt(bf16 v) { return __bfloat162float(v); }
+  static __device__ __forceinline__ void st(bf16* p, float v) { *p = __float2bfloat16_rn(v); }
+  static __device__ __forceinline__ void st64(bf16* p, double v) { *p = __double2bfloat16(v); }
+};
+
+template <typename T> __device__ __forceinline__ double to_f64(T v);
+template <> __device__ __forceinline__ double to_f64<float>(float v) { return (double)v; }
+template <> __device__ __forceinline__ double to_f64<bf16>(bf16 v) { return (double)__bfloat162float(v); }
+
+// ------------------------------------------------------------ reductions
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// RoPE inverse frequency of pair i for a rotary width d: theta^(-2i/d), in fp64.
+__device__ __forceinline__ double rope_inv_freq(double theta, int i, int d) {
+  return pow(theta, -2.0 * (double)i / (double)d);
+}
+
+// ------------------------------------------------------------ host helpers
+// Kernel launches issued by this library in this process (all devices).
+inline std::atomic<long long>& launch_counter() {
+  static std::atomic<long long> n{0};
+  return n;
+}
+static inline void note_launch(long long n = 1) { launch_counter().fetch_add(n, std::memory_order_relaxed); }
+
+static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+static inline int elem_bytes(const mla_config* cfg) { return cfg->dtype == MLA_BF16 ? 2 : 4; }
+
+static inline float scale_of(const mla_config* cfg) {
+  return cfg->softmax_scale > 0.f ? cfg->softmax_scale
+                                  : (float)(1.0 / sqrt((double)(cfg->qk_nope + cfg->d_r)));
+}
+
+}  // namespace mla

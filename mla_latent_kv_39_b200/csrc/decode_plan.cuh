@@ -1,0 +1,225 @@
+// Split-KV work plan shared by every decode kernel, and the split combine.
+//
+// The rows of all sequences, counted in cache pages, are laid end to end and
+// cut into `workers` contiguous, equally sized page ranges (+-1 page).  Where
+// a range crosses a sequence boundary it is cut again, so every piece - a
+// "segment" - covers pages [blk_begin, blk_end) of one sequence.  There are
+// at most workers + batch - 1 segments.  Each segment's decode writes, for
+// each of the sequence's n_q queries and each head, its output normalised
+// over its own rows plus the log2-sum-exp of its scaled scores; the combine
+// merges the segments of a sequence.  The plan is computed on the device
+// from seq_lens, so a decode step never waits on the host.
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+
+constexpr int kPlanMagic = 0x4D4C4131;  // "MLA1"
+
+struct DecodeLayout {
+  int batch, n_q, H, d_c, workers, max_segments;
+  long long off_prefix;        // int32 [batch + 1]   pages before sequence b
+  long long off_worker_first;  // int32 [workers + 1] first segment of worker w
+  long long off_seq_first;     // int32 [batch]       first segment of sequence b
+  long long off_seq_nseg;      // int32 [batch]       number of segments of sequence b
+  long long off_seg;           // int4  [max_segments] (b, blk_begin, blk_end, worker)
+  long long off_lse;           // f32   [max_segments, n_q, H]        log2-sum-exp
+  long long off_o;             // f32   [max_segments, n_q, H, d_c]   normalised partial output
+  long long total;
+};
+
+// Written by the plan kernel at offset 0 of the workspace; read by the combine.
+struct DecodeHeader {
+  int magic, batch, n_q, H, d_c, workers, max_segments, num_segments;
+  DecodeLayout layout;
+};
+
+static inline DecodeLayout decode_layout(int batch, int n_q, int H, int d_c, int workers) {
+  DecodeLayout L{};
+  L.batch = batch;
+  L.n_q = n_q;
+  L.H = H;
+  L.d_c = d_c;
+  L.workers = workers;
+  L.max_segments = workers + batch;
+  size_t o = align_up(sizeof(DecodeHeader), 256);
+  L.off_prefix = o;        o = align_up(o + sizeof(int) * (size_t)(batch + 1), 256);
+  L.off_worker_first = o;  o = align_up(o + sizeof(int) * (size_t)(workers + 1), 256);
+  L.off_seq_first = o;     o = align_up(o + sizeof(int) * (size_t)batch, 256);
+  L.off_seq_nseg = o;      o = align_up(o + sizeof(int) * (size_t)batch, 256);
+  L.off_seg = o;           o = align_up(o + sizeof(int4) * (size_t)L.max_segments, 256);
+  L.off_lse = o;           o = align_up(o + sizeof(float) * (size_t)L.max_segments * n_q * H, 256);
+  L.off_o = o;             o = align_up(o + sizeof(float) * (size_t)L.max_segments * n_q * H * d_c, 256);
+  L.total = o;
+  return L;
+}
+
+template <typename T> __device__ __forceinline__ T* ws_at(void* ws, long long off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+template <typename T> __device__ __forceinline__ const T* ws_at(const void* ws, long long off) {
+  return reinterpret_cast<const T*>(static_cast<const char*>(ws) + off);
+}
+
+// Exclusive prefix sum of value_of(0..n-1) into dst[0..n] (dst[n] = total), one CTA.
+template <typename F>
+__device__ int block_scan_exclusive(F value_of, int* dst, int n) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const int v = i < n ? value_of(i) : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      int w = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      if (lane < nw) warp_tot[lane] = w;
+    }
+    __syncthreads();
+    const int excl = carry + (wid > 0 ? warp_tot[wid - 1] : 0) + x - v;
+    if (i < n) dst[i] = excl;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = excl + v;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) dst[n] = carry;
+  __syncthreads();
+  return carry;
+}
+
+// Largest b in [0, batch) with P[b] <= g (requires 0 <= g < P[batch]).
+__device__ __forceinline__ int seq_of_page(const int* P, int batch, long long g) {
+  int lo = 0, hi = batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((long long)P[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __restrict__ seq_lens,
+                                                           int bs, int max_blocks, void* ws,
+                                                           DecodeLayout L) {
+  int* P = ws_at<int>(ws, L.off_prefix);
+  int* wfirst = ws_at<int>(ws, L.off_worker_first);
+  int* sfirst = ws_at<int>(ws, L.off_seq_first);
+  int* snseg = ws_at<int>(ws, L.off_seq_nseg);
+  int4* seg = ws_at<int4>(ws, L.off_seg);
+  const int batch = L.batch, n_q = L.n_q, W = L.workers;
+
+  auto pages_of = [&](int b) -> int {
+    const int len = seq_lens[b];
+    if (len < n_q || len > max_blocks * bs) {
+      report(MLA_ERR_BOUNDS, 4, b, len);
+      return 0;
+    }
+    return (len + bs - 1) / bs;
+  };
+  const int NB = block_scan_exclusive(pages_of, P, batch);
+
+  auto range_of = [&](int w, long long& s, long long& e) {
+    s = (long long)w * NB / W;
+    e = (long long)(w + 1) * NB / W;
+  };
+  auto segs_of = [&](int w) -> int {
+    long long s, e;
+    range_of(w, s, e);
+    if (s >= e) return 0;
+    return seq_of_page(P, batch, e - 1) - seq_of_page(P, batch, s) + 1;
+  };
+  const int nsegs = block_scan_exclusive(segs_of, wfirst, W);
+
+  for (int w = threadIdx.x; w < W; w += blockDim.x) {
+    long long s, e;
+    range_of(w, s, e);
+    if (s >= e) continue;
+    const int b0 = seq_of_page(P, batch, s), b1 = seq_of_page(P, batch, e - 1);
+    int k = wfirst[w];
+    for (int b = b0; b <= b1; ++b, ++k) {
+      const long long lo = s > P[b] ? s : P[b];
+      const long long hi = e < P[b + 1] ? e : P[b + 1];
+      seg[k] = make_int4(b, (int)(lo - P[b]), (int)(hi - P[b]), w);
+    }
+  }
+  for (int b = threadIdx.x; b < batch; b += blockDim.x) {
+    sfirst[b] = 0;
+    snseg[b] = 0;
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < nsegs; k += blockDim.x) {
+    const int b = seg[k].x;
+    if (k == 0 || seg[k - 1].x != b) sfirst[b] = k;
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < nsegs; k += blockDim.x) {
+    const int b = seg[k].x;
+    if (k == nsegs - 1 || seg[k + 1].x != b) snseg[b] = k - sfirst[b] + 1;
+  }
+  if (threadIdx.x == 0) {
+    DecodeHeader* h = ws_at<DecodeHeader>(ws, 0);
+    h->magic = kPlanMagic;
+    h->batch = batch;
+    h->n_q = n_q;
+    h->H = L.H;
+    h->d_c = L.d_c;
+    h->workers = W;
+    h->max_segments = L.max_segments;
+    h->num_segments = nsegs;
+    h->layout = L;
+  }
+}
+
+// o_lat[t, h, :] = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M) over the
+// segments of token t's sequence.  Grid (tokens, heads), block over d_c.
+__global__ void __launch_bounds__(128) combine_kernel(const void* ws, long long ws_bytes, int batch,
+                                                      int n_q, int H, int d_c, float* __restrict__ o_lat) {
+  const DecodeHeader* hd = ws_at<DecodeHeader>(ws, 0);
+  const int t = blockIdx.x, h = blockIdx.y;
+  float* out = o_lat + ((long long)t * H + h) * d_c;
+  if (hd->magic != kPlanMagic || hd->batch != batch || hd->n_q != n_q || hd->H != H ||
+      hd->d_c != d_c || hd->layout.total > ws_bytes) {
+    if (t == 0 && h == 0 && threadIdx.x == 0) report(MLA_ERR_WORKSPACE, 0, batch, n_q);
+    for (int d = threadIdx.x; d < d_c; d += blockDim.x) out[d] = 0.f;
+    return;
+  }
+  const DecodeLayout L = hd->layout;
+  const int b = t / n_q, j = t % n_q;
+  const int first = ws_at<int>(ws, L.off_seq_first)[b];
+  const int n = ws_at<int>(ws, L.off_seq_nseg)[b];
+  const float* lse = ws_at<float>(ws, L.off_lse);
+  const float* part = ws_at<float>(ws, L.off_o);
+  float M = -INFINITY;
+  for (int s = 0; s < n; ++s) M = fmaxf(M, lse[((long long)(first + s) * n_q + j) * H + h]);
+  if (n == 0 || M == -INFINITY) {
+    for (int d = threadIdx.x; d < d_c; d += blockDim.x) out[d] = 0.f;
+    return;
+  }
+  float Z = 0.f;
+  for (int s = 0; s < n; ++s) Z += exp2f(lse[((long long)(first + s) * n_q + j) * H + h] - M);
+  const float invZ = 1.f / Z;
+  for (int d = threadIdx.x; d < d_c; d += blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < n; ++s) {
+      const long long r = ((long long)(first + s) * n_q + j) * H + h;
+      acc += exp2f(lse[r] - M) * part[r * d_c + d];
+    }
+    out[d] = acc * invZ;
+  }
+}
+
+}  // namespace mla

@@ -1,0 +1,89 @@
+// Latent-space decode on CUDA cores: one warp per (segment, query, head).
+// Used for the fp32 storage path (small shapes, exact fp32 arithmetic).
+//
+// For its rows u of the segment (u <= the query's position p):
+//   s_u = (q_lat . c_u + q_R . kR_u) * scale * log2(e)
+// with an online (running-max) softmax, O = sum_u 2^(s_u - m) c_u / l.
+#pragma once
+
+#include "decode_plan.cuh"
+
+namespace mla {
+
+constexpr int kSimtDecodeMaxRow = 1024;  // d_c + d_r handled by one warp (32 lanes x 32 values)
+
+template <typename T, int DPL>
+__global__ void __launch_bounds__(128) decode_simt_kernel(
+    const T* __restrict__ q_lat, const T* __restrict__ q_rope, const T* __restrict__ pool,
+    const int32_t* __restrict__ block_table, int max_blocks, int num_blocks,
+    const int32_t* __restrict__ seq_lens, int n_q, int H, int d_c, int d_r, int bs,
+    float scale_log2, void* ws, DecodeLayout L) {
+  const DecodeHeader* hd = ws_at<DecodeHeader>(ws, 0);
+  const int sidx = blockIdx.x;
+  if (sidx >= hd->num_segments) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int idx = blockIdx.y * 4 + warp;
+  if (idx >= n_q * H) return;
+  const int j = idx / H, h = idx % H;
+  const int4 sg = ws_at<int4>(ws, L.off_seg)[sidx];
+  const int b = sg.x;
+  const int t = b * n_q + j;
+  const int p = seq_lens[b] - n_q + j;  // last row this query sees
+  const int row = d_c + d_r;
+
+  float q[DPL], o[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    const int d = lane + 32 * i;
+    float v = 0.f;
+    if (d < d_c) v = Store<T>::ld(q_lat + ((long long)t * H + h) * d_c + d);
+    else if (d < row) v = Store<T>::ld(q_rope + ((long long)t * H + h) * d_r + (d - d_c));
+    q[i] = v;
+    o[i] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  for (int blk = sg.y; blk < sg.z; ++blk) {
+    const int u0 = blk * bs;
+    const int nrows = min(bs, p + 1 - u0);
+    if (nrows <= 0) break;
+    const int phys = block_table[(long long)b * max_blocks + blk];
+    if (phys < 0 || phys >= num_blocks) {
+      if (lane == 0) report(MLA_ERR_BOUNDS, 5, b, phys);
+      continue;
+    }
+    const T* base = pool + (long long)phys * bs * row;
+    for (int r = 0; r < nrows; ++r) {
+      const T* kv = base + (long long)r * row;
+      float part = 0.f;
+      float c[DPL];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        const int d = lane + 32 * i;
+        c[i] = d < row ? Store<T>::ld(kv + d) : 0.f;
+        part = fmaf(q[i], c[i], part);
+      }
+      const float s = warp_sum(part) * scale_log2;
+      const float m_new = fmaxf(m, s);
+      const float corr = exp2f(m - m_new);
+      const float pw = exp2f(s - m_new);
+      l = l * corr + pw;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        const int d = lane + 32 * i;
+        o[i] = o[i] * corr + (d < d_c ? pw * c[i] : 0.f);
+      }
+      m = m_new;
+    }
+  }
+  const long long r_out = ((long long)sidx * n_q + j) * H + h;
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  float* out = ws_at<float>(ws, L.off_o) + r_out * d_c;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    const int d = lane + 32 * i;
+    if (d < d_c) out[d] = o[i] * inv;
+  }
+  if (lane == 0) ws_at<float>(ws, L.off_lse)[r_out] = l > 0.f ? m + log2f(l) : -INFINITY;
+}
+
+}  // namespace mla

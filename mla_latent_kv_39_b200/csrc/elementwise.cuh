@@ -1,0 +1,116 @@
+// Epilogue kernels of the projection steps: storage rounding, decoupled RoPE,
+// the paged-cache scatter of new latent rows, and the query split.
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+
+// Round an fp32 buffer to the storage type.
+template <typename T>
+__global__ void round_store_kernel(const float* __restrict__ src, T* __restrict__ dst, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    Store<T>::st(dst + i, src[i]);
+}
+
+template <typename T>
+static cudaError_t round_store(const float* src, T* dst, long long n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  int blocks = (int)std::min<long long>((n + 255) / 256, 4096);
+  round_store_kernel<T><<<blocks, 256, 0, s>>>(src, dst, n);
+  note_launch();
+  return cudaGetLastError();
+}
+
+// Where token t's cache row goes, or -1 after recording a bounds error.
+__device__ __forceinline__ long long cache_row_slot(const int32_t* seq_idx, const int32_t* pos, int t,
+                                                    const int32_t* block_table, int batch,
+                                                    int max_blocks, int num_blocks, int bs) {
+  const int b = seq_idx[t], p = pos[t];
+  if (b < 0 || b >= batch || p < 0) {
+    report(MLA_ERR_BOUNDS, 1, t, p);
+    return -1;
+  }
+  const int page = p / bs;
+  if (page >= max_blocks) {
+    report(MLA_ERR_BOUNDS, 2, t, p);
+    return -1;
+  }
+  const int phys = block_table[(long long)b * max_blocks + page];
+  if (phys < 0 || phys >= num_blocks) {
+    report(MLA_ERR_BOUNDS, 3, t, phys);
+    return -1;
+  }
+  return (long long)phys * bs + (p % bs);
+}
+
+// New latent rows from exact (fp64) projections C = x [W_DKV | W_KR]:
+// c = C[:, :d_c], k_R = RoPE(C[:, d_c:], pos); each value rounded once to T
+// and written to its paged slot.  One thread per latent value or rotary pair.
+template <typename T>
+__global__ void append_finish_kernel(const double* __restrict__ C, int n_tok, int d_c, int d_r,
+                                     double theta, const int32_t* __restrict__ seq_idx,
+                                     const int32_t* __restrict__ pos, T* __restrict__ pool,
+                                     const int32_t* __restrict__ block_table, int batch,
+                                     int max_blocks, int num_blocks, int bs) {
+  const int per_tok = d_c + d_r / 2;
+  const long long total = (long long)n_tok * per_tok;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(i / per_tok), k = (int)(i % per_tok);
+    const long long slot = cache_row_slot(seq_idx, pos, t, block_table, batch, max_blocks, num_blocks, bs);
+    if (slot < 0) continue;
+    const int row = d_c + d_r;
+    const double* src = C + (long long)t * row;
+    T* dst = pool + slot * row;
+    if (k < d_c) {
+      Store<T>::st64(dst + k, src[k]);
+    } else {
+      const int pr = k - d_c;  // rotary pair index
+      const double ang = (double)pos[t] * rope_inv_freq(theta, pr, d_r);
+      double sn, cs;
+      sincos(ang, &sn, &cs);
+      const double r0 = src[d_c + 2 * pr], r1 = src[d_c + 2 * pr + 1];
+      Store<T>::st64(dst + d_c + 2 * pr, r0 * cs - r1 * sn);
+      Store<T>::st64(dst + d_c + 2 * pr + 1, r0 * sn + r1 * cs);
+    }
+  }
+}
+
+// Split q [n, H, nope + d_r] (fp32) into q_nope (storage type) and the rotated
+// q_rope (storage type).  The RoPE angle and rotation are evaluated in fp64.
+template <typename T>
+__global__ void query_split_kernel(const float* __restrict__ q, int n_tok, int H, int nope, int d_r,
+                                   double theta, const int32_t* __restrict__ pos,
+                                   T* __restrict__ q_nope, T* __restrict__ q_rope) {
+  const int w = nope + d_r;
+  const int per_head = nope + d_r / 2;
+  const long long total = (long long)n_tok * H * per_head;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long th = i / per_head;  // t * H + h
+    const int k = (int)(i % per_head);
+    const int t = (int)(th / H);
+    const float* src = q + th * w;
+    if (k < nope) {
+      Store<T>::st(q_nope + th * nope + k, src[k]);
+    } else {
+      const int pr = k - nope;
+      const double ang = (double)pos[t] * rope_inv_freq(theta, pr, d_r);
+      double sn, cs;
+      sincos(ang, &sn, &cs);
+      const double r0 = src[nope + 2 * pr], r1 = src[nope + 2 * pr + 1];
+      Store<T>::st(q_rope + th * d_r + 2 * pr, (float)(r0 * cs - r1 * sn));
+      Store<T>::st(q_rope + th * d_r + 2 * pr + 1, (float)(r0 * sn + r1 * cs));
+    }
+  }
+}
+
+static inline int grid_for(long long n, int threads = 256, int cap = 8192) {
+  long long b = (n + threads - 1) / threads;
+  if (b < 1) b = 1;
+  return (int)(b > cap ? cap : b);
+}
+
+}  // namespace mla

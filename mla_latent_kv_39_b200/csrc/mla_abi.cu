@@ -1,0 +1,332 @@
+// C ABI of libmla.so: argument validation, workspace carving and launches.
+// Every step of the path runs in the kernels included below; this file only
+// checks arguments, computes workspace offsets and launches.
+#include <algorithm>
+#include <cmath>
+
+#include "common.cuh"
+#include "decode_plan.cuh"
+#include "decode_simt.cuh"
+#include "elementwise.cuh"
+#include "gemm_simt.cuh"
+
+using namespace mla;
+
+namespace {
+
+mla_status check_cfg(const mla_config* c) {
+  if (!c) return MLA_ERR_INVALID_ARG;
+  if (c->hidden <= 0 || c->n_heads <= 0 || c->d_c <= 0 || c->d_r <= 0 || c->qk_nope <= 0 ||
+      c->v_head <= 0 || c->q_lora < 0 || c->block_size <= 0 || (c->d_r & 1) ||
+      !(c->rope_theta > 0.0) || c->softmax_scale < 0.f)
+    return MLA_ERR_INVALID_ARG;
+  if (c->dtype != MLA_F32 && c->dtype != MLA_BF16) return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+
+mla_status check_cache(const mla_cache* k) {
+  if (!k || !k->pool || !k->block_table || k->num_blocks <= 0 || k->batch <= 0 ||
+      k->max_blocks_per_seq <= 0)
+    return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+
+inline mla_status st(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+#define MLA_TRY(expr)                          \
+  do {                                         \
+    mla_status _s = (expr);                    \
+    if (_s != MLA_OK) return _s;               \
+  } while (0)
+#define MLA_CUDA(expr) MLA_TRY(st(expr))
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+// ---------------------------------------------------------------- append
+size_t append_ws(const mla_config* c, int n_tok) {
+  return align_up(sizeof(double) * (size_t)n_tok * (c->d_c + c->d_r), 256);
+}
+
+template <typename T>
+mla_status append_impl(const mla_config* c, const void* x, int n, const void* W_DKV, const void* W_KR,
+                       const int32_t* seq_idx, const int32_t* pos, const mla_cache* k, void* ws,
+                       cudaStream_t s) {
+  const int row = c->d_c + c->d_r;
+  double* C = static_cast<double*>(ws);
+  MLA_CUDA((gemm_rm<T, double>(x, c->hidden, W_DKV, c->d_c, C, row, n, c->d_c, c->hidden, s)));
+  MLA_CUDA((gemm_rm<T, double>(x, c->hidden, W_KR, c->d_r, C + c->d_c, row, n, c->d_r, c->hidden, s)));
+  const long long total = (long long)n * (c->d_c + c->d_r / 2);
+  append_finish_kernel<T><<<grid_for(total), 256, 0, s>>>(
+      C, n, c->d_c, c->d_r, c->rope_theta, seq_idx, pos, static_cast<T*>(k->pool), k->block_table,
+      k->batch, k->max_blocks_per_seq, k->num_blocks, c->block_size);
+  note_launch();
+  return st(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------- absorb
+struct AbsorbWs {
+  size_t cq_f, cq_t, q_f, qn_t, ql_f, total;
+};
+AbsorbWs absorb_ws(const mla_config* c, int n) {
+  const size_t eb = elem_bytes(c);
+  const size_t H = c->n_heads, qw = H * (c->qk_nope + c->d_r);
+  AbsorbWs w{};
+  size_t o = 0;
+  w.cq_f = o; o = align_up(o + 4 * (size_t)n * c->q_lora, 256);
+  w.cq_t = o; o = align_up(o + eb * (size_t)n * c->q_lora, 256);
+  w.q_f = o;  o = align_up(o + 4 * (size_t)n * qw, 256);
+  w.qn_t = o; o = align_up(o + eb * (size_t)n * H * c->qk_nope, 256);
+  w.ql_f = o; o = align_up(o + 4 * (size_t)n * H * c->d_c, 256);
+  w.total = o;
+  return w;
+}
+
+template <typename T>
+mla_status absorb_impl(const mla_config* c, const void* x, int n, const void* W_DQ, const void* W_UQ,
+                       const void* W_UK, const int32_t* pos, void* q_lat, void* q_rope, void* ws,
+                       cudaStream_t s) {
+  const AbsorbWs w = absorb_ws(c, n);
+  char* base = static_cast<char*>(ws);
+  float* cq_f = reinterpret_cast<float*>(base + w.cq_f);
+  T* cq_t = reinterpret_cast<T*>(base + w.cq_t);
+  float* q_f = reinterpret_cast<float*>(base + w.q_f);
+  T* qn_t = reinterpret_cast<T*>(base + w.qn_t);
+  float* ql_f = reinterpret_cast<float*>(base + w.ql_f);
+  const int H = c->n_heads, nope = c->qk_nope, qw = H * (nope + c->d_r);
+  if (c->q_lora > 0) {
+    MLA_CUDA((gemm_rm<T, float>(x, c->hidden, W_DQ, c->q_lora, cq_f, c->q_lora, n, c->q_lora, c->hidden, s)));
+    MLA_CUDA(round_store<T>(cq_f, cq_t, (long long)n * c->q_lora, s));
+    MLA_CUDA((gemm_rm<T, float>(cq_t, c->q_lora, W_UQ, qw, q_f, qw, n, qw, c->q_lora, s)));
+  } else {
+    MLA_CUDA((gemm_rm<T, float>(x, c->hidden, W_UQ, qw, q_f, qw, n, qw, c->hidden, s)));
+  }
+  const long long tot = (long long)n * H * (nope + c->d_r / 2);
+  query_split_kernel<T><<<grid_for(tot), 256, 0, s>>>(q_f, n, H, nope, c->d_r, c->rope_theta, pos, qn_t,
+                                                      static_cast<T*>(q_rope));
+  note_launch();
+  MLA_CUDA(cudaGetLastError());
+  // q_lat[t, h, :] = q_nope[t, h, :] W_UK_h^T, batched over heads
+  GemmSimtArgs g{qn_t, W_UK, ql_f, n, c->d_c, nope, H,
+                 (long long)H * nope, 1, nope,
+                 1, (long long)H * nope, nope,
+                 (long long)H * c->d_c, 1, c->d_c};
+  MLA_CUDA((gemm_simt<T, float>(g, s)));
+  MLA_CUDA(round_store<T>(ql_f, static_cast<T*>(q_lat), (long long)n * H * c->d_c, s));
+  return MLA_OK;
+}
+
+// ---------------------------------------------------------------- out proj
+struct OutWs {
+  size_t ol_t, oh_f, oh_t, y_f, total;
+};
+OutWs out_ws(const mla_config* c, int n) {
+  const size_t eb = elem_bytes(c), H = c->n_heads;
+  OutWs w{};
+  size_t o = 0;
+  w.ol_t = o; o = align_up(o + eb * (size_t)n * H * c->d_c, 256);
+  w.oh_f = o; o = align_up(o + 4 * (size_t)n * H * c->v_head, 256);
+  w.oh_t = o; o = align_up(o + eb * (size_t)n * H * c->v_head, 256);
+  w.y_f = o;  o = align_up(o + 4 * (size_t)n * c->hidden, 256);
+  w.total = o;
+  return w;
+}
+
+template <typename T>
+mla_status out_impl(const mla_config* c, const float* o_lat, int n, const void* W_UV, const void* W_O,
+                    void* y, void* ws, cudaStream_t s) {
+  const OutWs w = out_ws(c, n);
+  char* base = static_cast<char*>(ws);
+  T* ol_t = reinterpret_cast<T*>(base + w.ol_t);
+  float* oh_f = reinterpret_cast<float*>(base + w.oh_f);
+  T* oh_t = reinterpret_cast<T*>(base + w.oh_t);
+  float* y_f = reinterpret_cast<float*>(base + w.y_f);
+  const int H = c->n_heads, dv = c->v_head;
+  MLA_CUDA(round_store<T>(o_lat, ol_t, (long long)n * H * c->d_c, s));
+  // o_h[t, h, :] = o_lat[t, h, :] W_UV_h, batched over heads
+  GemmSimtArgs g{ol_t, W_UV, oh_f, n, dv, c->d_c, H,
+                 (long long)H * c->d_c, 1, c->d_c,
+                 (long long)H * dv, 1, dv,
+                 (long long)H * dv, 1, dv};
+  MLA_CUDA((gemm_simt<T, float>(g, s)));
+  MLA_CUDA(round_store<T>(oh_f, oh_t, (long long)n * H * dv, s));
+  MLA_CUDA((gemm_rm<T, float>(oh_t, (long long)H * dv, W_O, c->hidden, y_f, c->hidden, n, c->hidden, H * dv, s)));
+  MLA_CUDA(round_store<T>(y_f, static_cast<T*>(y), (long long)n * c->hidden, s));
+  return MLA_OK;
+}
+
+// ---------------------------------------------------------------- decode
+int default_workers(const mla_config* c) {
+  const int sms = device_sm_count();
+  return std::max(1, 2 * (sms > 0 ? sms : 148));
+}
+
+int resolve_workers(const mla_config* c, int max_workers) {
+  return max_workers > 0 ? max_workers : default_workers(c);
+}
+
+template <typename T, int DPL>
+void launch_decode_simt(const mla_config* c, const void* q_lat, const void* q_rope, int n_q,
+                        const mla_cache* k, const int32_t* seq_lens, void* ws, const DecodeLayout& L,
+                        cudaStream_t s) {
+  const float scale_log2 = scale_of(c) * 1.4426950408889634f;
+  dim3 grid(L.max_segments, (n_q * c->n_heads + 3) / 4);
+  decode_simt_kernel<T, DPL><<<grid, 128, 0, s>>>(
+      static_cast<const T*>(q_lat), static_cast<const T*>(q_rope), static_cast<const T*>(k->pool),
+      k->block_table, k->max_blocks_per_seq, k->num_blocks, seq_lens, n_q, c->n_heads, c->d_c, c->d_r,
+      c->block_size, scale_log2, ws, L);
+  note_launch();
+}
+
+template <typename T>
+mla_status decode_simt_dispatch(const mla_config* c, const void* q_lat, const void* q_rope, int n_q,
+                                const mla_cache* k, const int32_t* seq_lens, void* ws,
+                                const DecodeLayout& L, cudaStream_t s) {
+  const int row = c->d_c + c->d_r;
+  if (row <= 96) launch_decode_simt<T, 3>(c, q_lat, q_rope, n_q, k, seq_lens, ws, L, s);
+  else if (row <= 576) launch_decode_simt<T, 18>(c, q_lat, q_rope, n_q, k, seq_lens, ws, L, s);
+  else if (row <= kSimtDecodeMaxRow) launch_decode_simt<T, 32>(c, q_lat, q_rope, n_q, k, seq_lens, ws, L, s);
+  else return MLA_ERR_UNSUPPORTED;
+  return st(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t mla_abi_version(void) { return MLA_ABI_VERSION; }
+
+int64_t mla_kernel_launches(void) { return launch_counter().load(std::memory_order_relaxed); }
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_INVALID_ARG: return "invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "unsupported dimensions";
+    case MLA_ERR_CUDA: return "CUDA error";
+    case MLA_ERR_BOUNDS: return "index out of bounds (device)";
+    case MLA_ERR_TIMEOUT: return "bounded wait timed out (device)";
+    case MLA_ERR_WORKSPACE: return "workspace too small or not written by mla_decode";
+  }
+  return "unknown status";
+}
+
+size_t mla_cache_append_workspace_size(const mla_config* cfg, int32_t n_tok) {
+  if (check_cfg(cfg) != MLA_OK || n_tok < 0) return 0;
+  return append_ws(cfg, n_tok);
+}
+
+mla_status mla_cache_append(const mla_config* cfg, const void* x, int32_t n_tok, const void* W_DKV,
+                            const void* W_KR, const int32_t* seq_idx, const int32_t* pos,
+                            const mla_cache* cache, void* workspace, size_t ws_bytes, void* stream) {
+  MLA_TRY(check_cfg(cfg));
+  if (n_tok < 0) return MLA_ERR_INVALID_ARG;
+  if (n_tok == 0) return MLA_OK;
+  if (!x || !W_DKV || !W_KR || !seq_idx || !pos || !workspace) return MLA_ERR_INVALID_ARG;
+  MLA_TRY(check_cache(cache));
+  if (ws_bytes < append_ws(cfg, n_tok)) return MLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cfg->dtype == MLA_BF16)
+    return append_impl<bf16>(cfg, x, n_tok, W_DKV, W_KR, seq_idx, pos, cache, workspace, s);
+  return append_impl<float>(cfg, x, n_tok, W_DKV, W_KR, seq_idx, pos, cache, workspace, s);
+}
+
+size_t mla_absorb_q_workspace_size(const mla_config* cfg, int32_t n_tok) {
+  if (check_cfg(cfg) != MLA_OK || n_tok < 0) return 0;
+  return absorb_ws(cfg, n_tok).total;
+}
+
+mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok, const void* W_DQ,
+                        const void* W_UQ, const void* W_UK, const int32_t* pos, void* q_lat,
+                        void* q_rope, void* workspace, size_t ws_bytes, void* stream) {
+  MLA_TRY(check_cfg(cfg));
+  if (n_tok < 0) return MLA_ERR_INVALID_ARG;
+  if (n_tok == 0) return MLA_OK;
+  if (!x || !W_UQ || !W_UK || !pos || !q_lat || !q_rope || !workspace) return MLA_ERR_INVALID_ARG;
+  if ((cfg->q_lora > 0) != (W_DQ != nullptr)) return MLA_ERR_INVALID_ARG;
+  if (ws_bytes < absorb_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cfg->dtype == MLA_BF16)
+    return absorb_impl<bf16>(cfg, x, n_tok, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, workspace, s);
+  return absorb_impl<float>(cfg, x, n_tok, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, workspace, s);
+}
+
+size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t n_q, int32_t max_workers) {
+  if (check_cfg(cfg) != MLA_OK || batch < 0 || n_q <= 0 || max_workers < 0) return 0;
+  return (size_t)decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers)).total;
+}
+
+mla_status mla_decode(const mla_config* cfg, const void* q_lat, const void* q_rope, int32_t batch,
+                      int32_t n_q, const mla_cache* cache, const int32_t* seq_lens, int32_t max_workers,
+                      void* workspace, size_t ws_bytes, void* stream) {
+  MLA_TRY(check_cfg(cfg));
+  if (batch < 0 || n_q <= 0 || max_workers < 0) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!q_lat || !q_rope || !seq_lens || !workspace) return MLA_ERR_INVALID_ARG;
+  MLA_TRY(check_cache(cache));
+  if (cache->batch < batch) return MLA_ERR_INVALID_ARG;
+  const DecodeLayout L =
+      decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers));
+  if (ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  decode_plan_kernel<<<1, 1024, 0, s>>>(seq_lens, cfg->block_size, cache->max_blocks_per_seq, workspace, L);
+  note_launch();
+  MLA_CUDA(cudaGetLastError());
+  if (cfg->dtype == MLA_BF16)
+    return decode_simt_dispatch<bf16>(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, s);
+  return decode_simt_dispatch<float>(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, s);
+}
+
+mla_status mla_combine(const mla_config* cfg, const void* workspace, size_t ws_bytes, int32_t batch,
+                       int32_t n_q, float* o_lat, void* stream) {
+  MLA_TRY(check_cfg(cfg));
+  if (batch < 0 || n_q <= 0) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!workspace || !o_lat) return MLA_ERR_INVALID_ARG;
+  if (ws_bytes < sizeof(DecodeHeader)) return MLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dim3 grid(batch * n_q, cfg->n_heads);
+  combine_kernel<<<grid, 128, 0, s>>>(workspace, (long long)ws_bytes, batch, n_q, cfg->n_heads, cfg->d_c, o_lat);
+  note_launch();
+  return st(cudaGetLastError());
+}
+
+size_t mla_out_proj_workspace_size(const mla_config* cfg, int32_t n_tok) {
+  if (check_cfg(cfg) != MLA_OK || n_tok < 0) return 0;
+  return out_ws(cfg, n_tok).total;
+}
+
+mla_status mla_out_proj(const mla_config* cfg, const float* o_lat, int32_t n_tok, const void* W_UV,
+                        const void* W_O, void* y, void* workspace, size_t ws_bytes, void* stream) {
+  MLA_TRY(check_cfg(cfg));
+  if (n_tok < 0) return MLA_ERR_INVALID_ARG;
+  if (n_tok == 0) return MLA_OK;
+  if (!o_lat || !W_UV || !W_O || !y || !workspace) return MLA_ERR_INVALID_ARG;
+  if (ws_bytes < out_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cfg->dtype == MLA_BF16) return out_impl<bf16>(cfg, o_lat, n_tok, W_UV, W_O, y, workspace, s);
+  return out_impl<float>(cfg, o_lat, n_tok, W_UV, W_O, y, workspace, s);
+}
+
+mla_status mla_get_device_error(void* stream, int32_t* detail) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MLA_ERR_CUDA;
+  int h[4] = {0, 0, 0, 0};
+  if (cudaMemcpyFromSymbol(h, g_err, sizeof(h)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (h[0] != 0) {
+    const int zero[4] = {0, 0, 0, 0};
+    if (cudaMemcpyToSymbol(g_err, zero, sizeof(zero)) != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  if (detail) {
+    detail[0] = h[1];
+    detail[1] = h[2];
+    detail[2] = h[3];
+  }
+  return static_cast<mla_status>(h[0]);
+}
+
+}  // extern "C"

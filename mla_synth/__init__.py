@@ -16,4 +16,5 @@ from .workloads import (  # noqa: F401
     generate,
     reduced,
     build_pool,
+    device_inputs,
 )

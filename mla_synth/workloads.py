@@ -297,6 +297,8 @@ def build_pool(data: WorkloadData, rows: Optional[torch.Tensor] = None,
     src = data.cached_rows if rows is None else rows
     pool = torch.full((max(data.num_blocks, 1), bs, shape.row), fill, dtype=shape.torch_dtype)
     flat = pool.view(-1, shape.row)
+    if src is None:          # rows are produced later by the append step
+        return pool
     for b in range(wl.batch):
         L = int(data.cached_len[b])
         if L == 0:
@@ -307,3 +309,25 @@ def build_pool(data: WorkloadData, rows: Optional[torch.Tensor] = None,
         s = int(data.row_offsets[b])
         flat[dst] = src[s:s + L]
     return pool
+
+
+def device_inputs(data: WorkloadData, device, pool: Optional[torch.Tensor] = None) -> Dict[str, object]:
+    """Copies of the seeded inputs on ``device`` (pure data movement)."""
+    dev = torch.device(device)
+    out: Dict[str, object] = {
+        "weights": {k: v.to(dev) for k, v in data.weights.items()},
+        "pool": (build_pool(data) if pool is None else pool).to(dev),
+        "block_table": data.block_table.to(dev),
+        "seq_lens": data.seq_lens.to(torch.int32).to(dev),
+        "x_new": data.x_new.to(dev),
+        "pos": data.new_positions().to(dev),
+        "seq_idx": data.new_seq_idx().to(dev),
+    }
+    if data.x_cached is not None:
+        L = int(data.cached_len.sum())
+        out["x_cached"] = data.x_cached.to(dev)
+        out["pos_cached"] = torch.cat([torch.arange(int(n), dtype=torch.int32)
+                                       for n in data.cached_len]).to(dev) if L else None
+        out["seq_idx_cached"] = torch.arange(data.workload.batch, dtype=torch.int32).repeat_interleave(
+            data.cached_len).to(dev)
+    return out

@@ -1,0 +1,125 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+symbol the header declares, its structs have the header's layout, and the
+synchronous argument checks answer before any launch."""
+
+import ctypes
+import re
+import subprocess
+from pathlib import Path
+
+import pytest
+
+from mla_latent_kv_39_b200 import abi, build
+
+ROOT = Path(__file__).resolve().parents[1]
+HEADER = ROOT / "include" / "mla.h"
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return abi.load_library()
+
+
+def declared_functions():
+    text = re.sub(r"/\*.*?\*/", "", HEADER.read_text(), flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_five_steps():
+    names = declared_functions()
+    for step in ("mla_cache_append", "mla_absorb_q", "mla_decode", "mla_combine", "mla_out_proj"):
+        assert step in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", str(abi._LIB_PATH)], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\b(mla_[a-z0-9_]+)\b", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    assert set(abi.SIGNATURES) == set(declared_functions())
+
+
+def test_struct_layout_matches_the_header(tmp_path):
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "mla.h"\n'
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu\\n\", sizeof(mla_config),"
+        " offsetof(mla_config, rope_theta), offsetof(mla_config, dtype), sizeof(mla_cache),"
+        " offsetof(mla_cache, block_table), offsetof(mla_cache, max_blocks_per_seq));return 0;}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", f"-I{ROOT / 'include'}", str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    want = [ctypes.sizeof(abi.MLAConfig), abi.MLAConfig.rope_theta.offset, abi.MLAConfig.dtype.offset,
+            ctypes.sizeof(abi.MLACache), abi.MLACache.block_table.offset,
+            abi.MLACache.max_blocks_per_seq.offset]
+    assert got == want
+
+
+def _cfg(**kw):
+    base = dict(hidden=256, n_heads=4, d_c=64, d_r=16, qk_nope=32, v_head=32, q_lora=0, dtype="f32")
+    base.update(kw)
+    return abi.Config(**base).c()
+
+
+def test_abi_version(lib):
+    assert lib.mla_abi_version() == 1
+
+
+def test_invalid_configs_are_rejected_synchronously(lib):
+    P = ctypes.byref
+    assert lib.mla_cache_append(None, None, 1, None, None, None, None, None, None, 0, None) == abi.MLA_ERR_INVALID_ARG
+    for bad in (dict(d_r=15), dict(n_heads=0), dict(block_size=0), dict(dtype=7), dict(rope_theta=0.0)):
+        if "dtype" in bad:
+            c = _cfg()
+            c.dtype = bad["dtype"]
+        else:
+            c = _cfg(**bad)
+        assert lib.mla_decode_workspace_size(P(c), 1, 1, 0) == 0
+        assert lib.mla_out_proj(P(c), None, 1, None, None, None, None, 0, None) == abi.MLA_ERR_INVALID_ARG
+
+
+def test_null_pointers_and_small_workspace_answer_before_launch(lib):
+    P = ctypes.byref
+    c = _cfg()
+    fake = ctypes.c_void_p(0x1000)   # never dereferenced: every check below fails first
+    assert lib.mla_absorb_q(P(c), None, 2, None, fake, fake, fake, fake, fake, fake, 1 << 20, None) \
+        == abi.MLA_ERR_INVALID_ARG
+    # W_DQ given although q_lora == 0
+    assert lib.mla_absorb_q(P(c), fake, 2, fake, fake, fake, fake, fake, fake, fake, 1 << 20, None) \
+        == abi.MLA_ERR_INVALID_ARG
+    need = lib.mla_out_proj_workspace_size(P(c), 5)
+    assert need > 0
+    assert lib.mla_out_proj(P(c), fake, 5, fake, fake, fake, fake, need - 1, None) == abi.MLA_ERR_WORKSPACE
+    cache = abi.MLACache(0x2000, 4, 0x3000, 1, 2)
+    need = lib.mla_decode_workspace_size(P(c), 1, 1, 8)
+    assert lib.mla_decode(P(c), fake, fake, 1, 1, P(cache), fake, 8, fake, need - 1, None) == abi.MLA_ERR_WORKSPACE
+    assert lib.mla_decode(P(c), fake, fake, 2, 1, P(cache), fake, 8, fake, need, None) == abi.MLA_ERR_INVALID_ARG
+    assert lib.mla_decode(P(c), fake, fake, 1, 0, P(cache), fake, 8, fake, need, None) == abi.MLA_ERR_INVALID_ARG
+
+
+def test_empty_work_is_a_no_op(lib):
+    P = ctypes.byref
+    c = _cfg()
+    assert lib.mla_cache_append(P(c), None, 0, None, None, None, None, None, None, 0, None) == abi.MLA_OK
+    assert lib.mla_absorb_q(P(c), None, 0, None, None, None, None, None, None, None, 0, None) == abi.MLA_OK
+    assert lib.mla_decode(P(c), None, None, 0, 1, None, None, 0, None, 0, None) == abi.MLA_OK
+    assert lib.mla_combine(P(c), None, 0, 0, 1, None, None) == abi.MLA_OK
+    assert lib.mla_out_proj(P(c), None, 0, None, None, None, None, 0, None) == abi.MLA_OK
+
+
+def test_decode_workspace_grows_with_workers_and_batch(lib):
+    P = ctypes.byref
+    c = _cfg(hidden=7168, n_heads=128, d_c=512, d_r=64, qk_nope=128, v_head=128, q_lora=1536, dtype="bf16")
+    a = lib.mla_decode_workspace_size(P(c), 64, 1, 74)
+    b = lib.mla_decode_workspace_size(P(c), 64, 1, 148)
+    d = lib.mla_decode_workspace_size(P(c), 64, 2, 74)
+    seg_bytes = 128 * 512 * 4
+    assert b - a >= 74 * seg_bytes and d - a >= (74 + 64) * seg_bytes
+
+
+def test_status_strings(lib):
+    for code in range(-6, 1):
+        assert lib.mla_status_string(code)

@@ -1,0 +1,148 @@
+"""CUDA path vs the fp64 oracle, through the C ABI, on seeded inputs.
+
+Small cases compare every output element; full-size workloads (the same
+launch configuration the benchmark times) compare sampled sequences, which
+the oracle computes one by one in the absorbed order (itself pinned to the
+decompressed order to 1e-10).  The cache rows that a step appends must be
+bit-identical to the oracle's once-rounded rows.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mla_synth import WORKLOADS, build_pool, generate, reduced
+from mla_latent_kv_39_b200 import (MLAError, Cache, Config, DecodeLayer, abi, check_device_error,
+                                   mla_get_device_error)
+
+from mla_gpu_cases import (check_new_cache_rows, check_outputs, oracle_expect, pool_row, run_gpu,
+                           tol_for, assert_close)
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_fp32_whole_config():
+    wl = WORKLOADS["tiny_f32_b1_l128"]
+    data, dev, layer = run_gpu(wl)
+    exp = oracle_expect(data, order="decompressed")
+    exp_abs = oracle_expect(data, order="absorbed")
+    # every cached row (appended by the library from x_cached) is exact
+    for p in range(int(data.cached_len[0])):
+        want = np.concatenate([exp["cached_c"][0][p], exp["cached_kr"][0][p]])
+        assert np.array_equal(pool_row(layer, data, 0, p), want), p
+    check_new_cache_rows(layer, data, exp)
+    exp["o_lat"] = exp_abs["o_lat"]
+    check_outputs(layer, data, exp, range(wl.n_tok))
+
+
+SMALL_CASES = [
+    # name, reduced lengths, n_q  (page-boundary, single-row and long rows)
+    ("v2_b16_l4096", [4096, 63, 64, 65, 0], None),
+    ("v3_b64_ragged1k_8k", [700, 1, 130, 191, 257, 64], None),
+    ("v3_b4_long", [5000, 20000], None),
+    ("v3_b128_nq2_ragged512_16k", [0, 1, 62, 63, 64, 300], 2),
+]
+
+
+@pytest.mark.parametrize("name,lengths,n_q", SMALL_CASES, ids=[c[0] for c in SMALL_CASES])
+def test_small_cases_every_element(name, lengths, n_q):
+    wl = reduced(WORKLOADS[name], lengths=lengths, n_q=n_q)
+    data, dev, layer = run_gpu(wl)
+    exp = oracle_expect(data, order="decompressed")
+    exp_abs = oracle_expect(data, order="absorbed")
+    check_new_cache_rows(layer, data, exp)
+    exp["o_lat"] = exp_abs["o_lat"]
+    check_outputs(layer, data, exp, range(wl.n_tok))
+
+
+FULL = ["v2_b16_l4096", "v3_b64_ragged1k_8k", "v3_b4_long", "v3_b128_nq2_ragged512_16k"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(name):
+    wl = WORKLOADS[name]
+    data, dev, layer = run_gpu(wl)
+    L = data.cached_len.numpy()
+    seqs = sorted({int(np.argmin(L)), int(np.argmax(L)), wl.batch // 2})
+    exp = oracle_expect(data, seqs=seqs, order="absorbed")
+    check_new_cache_rows(layer, data, exp)
+    toks = [b * wl.n_q + j for b in seqs for j in range(wl.n_q)]
+    check_outputs(layer, data, exp, toks)
+
+
+def test_split_count_does_not_change_the_result():
+    wl = reduced(WORKLOADS["v3_b64_ragged1k_8k"], lengths=[3000, 70, 1500])
+    data = generate(wl)
+    outs = []
+    for workers in (1, 3, 7, 0):
+        _, _, layer = run_gpu(wl, data=data, max_workers=workers)
+        outs.append(layer.o_lat.cpu().double().numpy())
+    for o in outs[1:]:
+        assert np.max(np.abs(o - outs[0])) <= 1e-5 * np.max(np.abs(outs[0]))
+
+
+def test_physical_page_order_does_not_change_the_result():
+    wl = reduced(WORKLOADS["v3_b64_ragged1k_8k"], lengths=[900, 333])
+    a = generate(wl)
+    _, _, la = run_gpu(wl, data=a)
+    # same logical rows, pages placed in reverse physical order
+    b = generate(wl)
+    b.block_table = torch.where(b.block_table >= 0, b.num_blocks - 1 - b.block_table, b.block_table)
+    _, _, lb = run_gpu(wl, data=b)
+    assert torch.equal(la.o_lat, lb.o_lat)
+    assert torch.equal(la.y, lb.y)
+
+
+def test_bad_block_id_is_reported_not_faulted():
+    wl = reduced(WORKLOADS["v3_b64_ragged1k_8k"], lengths=[200, 100])
+    data = generate(wl)
+    data.block_table[1, 0] = data.num_blocks + 5      # outside the pool
+    with pytest.raises(MLAError) as e:
+        run_gpu(wl, data=data)
+    assert e.value.status == abi.MLA_ERR_BOUNDS
+    assert mla_get_device_error()[0] == abi.MLA_OK    # cleared by the first read
+
+
+def test_sequence_shorter_than_its_queries_is_reported():
+    wl = reduced(WORKLOADS["v3_b128_nq2_ragged512_16k"], lengths=[10, 20], n_q=2)
+    data = generate(wl)
+    _, dev, layer = run_gpu(wl, data=data)
+    bad = dev["seq_lens"].clone()
+    bad[0] = 1
+    layer.attend(bad)
+    status, detail = mla_get_device_error()
+    assert status == abi.MLA_ERR_BOUNDS and detail[1] == 0
+    assert torch.count_nonzero(layer.o_lat[0:2]) == 0     # that sequence's output is zero
+    assert torch.count_nonzero(layer.o_lat[2:4]) > 0
+
+
+def test_combine_rejects_a_workspace_decode_never_wrote():
+    wl = reduced(WORKLOADS["v2_b16_l4096"], lengths=[64])
+    _, dev, layer = run_gpu(wl)
+    layer.ws_decode.zero_()
+    abi.mla_combine(layer.cfg, layer.ws_decode, 1, 1, layer.o_lat)
+    status, _ = mla_get_device_error()
+    assert status == abi.MLA_ERR_WORKSPACE
+    assert torch.count_nonzero(layer.o_lat) == 0
+
+
+def test_workspace_too_small_raises_before_launch():
+    wl = reduced(WORKLOADS["v2_b16_l4096"], lengths=[64])
+    _, dev, layer = run_gpu(wl)
+    with pytest.raises(MLAError) as e:
+        abi.mla_decode(layer.cfg, layer.q_lat, layer.q_rope, 1, 1, layer.cache, dev["seq_lens"],
+                       layer.ws_decode[:100], 0)
+    assert e.value.status == abi.MLA_ERR_WORKSPACE
+
+
+def test_empty_batch_is_a_no_op():
+    wl = reduced(WORKLOADS["v2_b16_l4096"], lengths=[64])
+    _, dev, layer = run_gpu(wl)
+    cfg = layer.cfg
+    H = cfg.n_heads
+    e = torch.empty(0, H, cfg.d_c, dtype=torch.bfloat16, device="cuda")
+    abi.mla_decode(cfg, e, torch.empty(0, H, cfg.d_r, dtype=torch.bfloat16, device="cuda"), 0, 1,
+                   layer.cache, torch.empty(0, dtype=torch.int32, device="cuda"), layer.ws_decode, 0)
+    torch.cuda.synchronize()
+    check_device_error()
