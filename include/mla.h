@@ -77,7 +77,14 @@ typedef struct {
   float softmax_scale;   /* 0 -> 1/sqrt(qk_nope + d_r) */
   int32_t block_size;    /* tokens per cache page */
   int32_t dtype;         /* mla_dtype */
+  int32_t flags;         /* OR of MLA_FLAG_* */
 } mla_config;
+
+/* Decode with the query held as a bf16 hi + lo pair on the tensor cores
+ * (about 16 significant bits instead of 8), for strongly peaked softmaxes
+ * where a bf16 query alone perturbs the dominant probabilities by ~1%.
+ * Costs extra score work in the bf16 decode kernel; no effect on fp32 storage. */
+#define MLA_FLAG_SPLIT_QUERY 1
 
 /* Paged latent cache of one layer ([P2] "MLA ve diğer optimizasyonlarla ilişkisi").
  * pool:        [num_blocks, block_size, d_c + d_r] storage dtype; row = [c_KV | k_R].
@@ -126,13 +133,15 @@ mla_status mla_cache_append(const mla_config* cfg, const void* x, int32_t n_tok,
  *   q_lat_h = q_nope_h W_UK_h^T  with  W_UK_h = W_UK[:, h qk_nope : (h+1) qk_nope].
  *   x      [n_tok, hidden];  W_DQ [hidden, q_lora];  W_UQ [q_lora or hidden, H (qk_nope + d_r)]
  *   W_UK   [d_c, H qk_nope];  pos int32 [n_tok]
- *   q_lat  [n_tok, H, d_c] (out, storage dtype);  q_rope [n_tok, H, d_r] (out)
+ *   q_lat  float32 [n_tok, H, d_c] (out);  q_rope float32 [n_tok, H, d_r] (out)
+ *   The query side keeps fp32 intermediates (c_Q, q, q_nope) and fp32
+ *   outputs: a bf16 query perturbs strongly peaked softmaxes by ~1%.
  *   workspace >= mla_absorb_q_workspace_size(cfg, n_tok) bytes
  * ------------------------------------------------------------------------- */
 size_t mla_absorb_q_workspace_size(const mla_config* cfg, int32_t n_tok);
 mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok,
                         const void* W_DQ, const void* W_UQ, const void* W_UK,
-                        const int32_t* pos, void* q_lat, void* q_rope,
+                        const int32_t* pos, float* q_lat, float* q_rope,
                         void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
@@ -147,7 +156,8 @@ mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok,
  * scheduled worker; each range writes an unnormalised-free partial
  * (softmax-normalised over its rows) and its log2-sum-exp into `workspace`;
  * mla_combine merges them.
- *   q_lat [batch n_q, H, d_c], q_rope [batch n_q, H, d_r]: from mla_absorb_q
+ *   q_lat float32 [batch n_q, H, d_c], q_rope float32 [batch n_q, H, d_r]:
+ *            from mla_absorb_q (row v = b n_q + j)
  *   seq_lens int32 [batch]: rows of each sequence INCLUDING the n_q new rows
  *            (already appended); must satisfy n_q <= seq_lens[b] <=
  *            max_blocks_per_seq * block_size.
@@ -158,7 +168,7 @@ mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok,
  * ------------------------------------------------------------------------- */
 size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t n_q,
                                  int32_t max_workers);
-mla_status mla_decode(const mla_config* cfg, const void* q_lat, const void* q_rope,
+mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_rope,
                       int32_t batch, int32_t n_q, const mla_cache* cache,
                       const int32_t* seq_lens, int32_t max_workers,
                       void* workspace, size_t ws_bytes, void* stream);

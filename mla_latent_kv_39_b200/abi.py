@@ -28,6 +28,7 @@ MLA_ERR_TIMEOUT = -5
 MLA_ERR_WORKSPACE = -6
 MLA_F32 = 0
 MLA_BF16 = 1
+MLA_FLAG_SPLIT_QUERY = 1
 
 # Every symbol the header declares, with (restype, argtypes).
 _vp, _i32, _sz, _d, _f = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_double, ctypes.c_float
@@ -39,7 +40,7 @@ class MLAConfig(ctypes.Structure):
     _fields_ = [("hidden", _i32), ("n_heads", _i32), ("d_c", _i32), ("d_r", _i32),
                 ("qk_nope", _i32), ("v_head", _i32), ("q_lora", _i32),
                 ("rope_theta", _d), ("softmax_scale", _f), ("block_size", _i32),
-                ("dtype", _i32)]
+                ("dtype", _i32), ("flags", _i32)]
 
 
 class MLACache(ctypes.Structure):
@@ -119,12 +120,13 @@ class Config:
     softmax_scale: float = 0.0
     block_size: int = 64
     dtype: str = "bf16"
+    split_query: bool = False
 
     @staticmethod
-    def from_shape(shape) -> "Config":
+    def from_shape(shape, split_query: bool = False) -> "Config":
         return Config(shape.hidden, shape.n_heads, shape.d_c, shape.d_r, shape.qk_nope,
                       shape.v_head, shape.q_lora, float(shape.rope_theta), 0.0,
-                      shape.block_size, shape.dtype)
+                      shape.block_size, shape.dtype, split_query)
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -133,7 +135,8 @@ class Config:
     def c(self) -> MLAConfig:
         return MLAConfig(self.hidden, self.n_heads, self.d_c, self.d_r, self.qk_nope, self.v_head,
                          self.q_lora, self.rope_theta, self.softmax_scale, self.block_size,
-                         MLA_BF16 if self.dtype == "bf16" else MLA_F32)
+                         MLA_BF16 if self.dtype == "bf16" else MLA_F32,
+                         MLA_FLAG_SPLIT_QUERY if self.split_query else 0)
 
 
 class Cache:
@@ -222,8 +225,8 @@ def mla_absorb_q(cfg: Config, x, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, workspace
         _need(W_UQ, "W_Q", dt, shape=(cfg.hidden, H * (cfg.qk_nope + cfg.d_r)))
     _need(W_UK, "W_UK", dt, shape=(cfg.d_c, H * cfg.qk_nope))
     _need(pos, "pos", torch.int32, shape=(n,))
-    _need(q_lat, "q_lat", dt, shape=(n, H, cfg.d_c))
-    _need(q_rope, "q_rope", dt, shape=(n, H, cfg.d_r))
+    _need(q_lat, "q_lat", torch.float32, shape=(n, H, cfg.d_c))
+    _need(q_rope, "q_rope", torch.float32, shape=(n, H, cfg.d_r))
     _need(workspace, "workspace", torch.uint8)
     _check(lib().mla_absorb_q(ctypes.byref(cfg.c()), _ptr(x), n, _ptr(W_DQ), _ptr(W_UQ), _ptr(W_UK),
                               _ptr(pos), _ptr(q_lat), _ptr(q_rope), _ptr(workspace), workspace.numel(),
@@ -234,8 +237,8 @@ def mla_decode(cfg: Config, q_lat, q_rope, batch: int, n_q: int, cache: Cache, s
                max_workers: int = 0, stream=None):
     dt = cfg.torch_dtype
     H = cfg.n_heads
-    _need(q_lat, "q_lat", dt, shape=(batch * n_q, H, cfg.d_c))
-    _need(q_rope, "q_rope", dt, shape=(batch * n_q, H, cfg.d_r))
+    _need(q_lat, "q_lat", torch.float32, shape=(batch * n_q, H, cfg.d_c))
+    _need(q_rope, "q_rope", torch.float32, shape=(batch * n_q, H, cfg.d_r))
     _need(seq_lens, "seq_lens", torch.int32, shape=(batch,))
     _need(workspace, "workspace", torch.uint8)
     _check(lib().mla_decode(ctypes.byref(cfg.c()), _ptr(q_lat), _ptr(q_rope), batch, n_q,

@@ -1,14 +1,17 @@
 // Split-KV work plan shared by every decode kernel, and the split combine.
 //
-// The rows of all sequences, counted in cache pages, are laid end to end and
-// cut into `workers` contiguous, equally sized page ranges (+-1 page).  Where
-// a range crosses a sequence boundary it is cut again, so every piece - a
-// "segment" - covers pages [blk_begin, blk_end) of one sequence.  There are
-// at most workers + batch - 1 segments.  Each segment's decode writes, for
-// each of the sequence's n_q queries and each head, its output normalised
-// over its own rows plus the log2-sum-exp of its scaled scores; the combine
-// merges the segments of a sequence.  The plan is computed on the device
-// from seq_lens, so a decode step never waits on the host.
+// The unit of work is a query row v = b * n_q + j (query j of sequence b).
+// Row v sees the cache rows 0 .. len_v - 1 of sequence b, with
+// len_v = seq_lens[b] - n_q + j + 1 (causal, its own row included), i.e.
+// ceil(len_v / block) pages.  The pages of all query rows, laid end to end,
+// are cut into `workers` contiguous, equally sized ranges (+-1 page); where a
+// range crosses a row boundary it is cut again, so every piece - a
+// "segment" - covers pages [blk_begin, blk_end) of one query row.  There are
+// at most workers + rows - 1 segments.  Each segment's decode writes, per
+// head, its output normalised over its own rows plus the log2-sum-exp of its
+// scaled scores; the combine merges the segments of a row.  The plan is
+// computed on the device from seq_lens, so a decode step never waits on the
+// host.
 #pragma once
 
 #include "common.cuh"
@@ -19,13 +22,13 @@ constexpr int kPlanMagic = 0x4D4C4131;  // "MLA1"
 
 struct DecodeLayout {
   int batch, n_q, H, d_c, workers, max_segments;
-  long long off_prefix;        // int32 [batch + 1]   pages before sequence b
+  long long off_prefix;        // int32 [rows + 1]    pages before query row v
   long long off_worker_first;  // int32 [workers + 1] first segment of worker w
-  long long off_seq_first;     // int32 [batch]       first segment of sequence b
-  long long off_seq_nseg;      // int32 [batch]       number of segments of sequence b
-  long long off_seg;           // int4  [max_segments] (b, blk_begin, blk_end, worker)
-  long long off_lse;           // f32   [max_segments, n_q, H]        log2-sum-exp
-  long long off_o;             // f32   [max_segments, n_q, H, d_c]   normalised partial output
+  long long off_seq_first;     // int32 [rows]        first segment of query row v
+  long long off_seq_nseg;      // int32 [rows]        number of segments of query row v
+  long long off_seg;           // int4  [max_segments] (v, blk_begin, blk_end, worker)
+  long long off_lse;           // f32   [max_segments, H]        log2-sum-exp
+  long long off_o;             // f32   [max_segments, H, d_c]   normalised partial output
   long long total;
 };
 
@@ -37,20 +40,21 @@ struct DecodeHeader {
 
 static inline DecodeLayout decode_layout(int batch, int n_q, int H, int d_c, int workers) {
   DecodeLayout L{};
+  const size_t rows = (size_t)batch * n_q;
   L.batch = batch;
   L.n_q = n_q;
   L.H = H;
   L.d_c = d_c;
   L.workers = workers;
-  L.max_segments = workers + batch;
+  L.max_segments = workers + (int)rows;
   size_t o = align_up(sizeof(DecodeHeader), 256);
-  L.off_prefix = o;        o = align_up(o + sizeof(int) * (size_t)(batch + 1), 256);
+  L.off_prefix = o;        o = align_up(o + sizeof(int) * (rows + 1), 256);
   L.off_worker_first = o;  o = align_up(o + sizeof(int) * (size_t)(workers + 1), 256);
-  L.off_seq_first = o;     o = align_up(o + sizeof(int) * (size_t)batch, 256);
-  L.off_seq_nseg = o;      o = align_up(o + sizeof(int) * (size_t)batch, 256);
+  L.off_seq_first = o;     o = align_up(o + sizeof(int) * rows, 256);
+  L.off_seq_nseg = o;      o = align_up(o + sizeof(int) * rows, 256);
   L.off_seg = o;           o = align_up(o + sizeof(int4) * (size_t)L.max_segments, 256);
-  L.off_lse = o;           o = align_up(o + sizeof(float) * (size_t)L.max_segments * n_q * H, 256);
-  L.off_o = o;             o = align_up(o + sizeof(float) * (size_t)L.max_segments * n_q * H * d_c, 256);
+  L.off_lse = o;           o = align_up(o + sizeof(float) * (size_t)L.max_segments * H, 256);
+  L.off_o = o;             o = align_up(o + sizeof(float) * (size_t)L.max_segments * H * d_c, 256);
   L.total = o;
   return L;
 }
@@ -102,9 +106,9 @@ __device__ int block_scan_exclusive(F value_of, int* dst, int n) {
   return carry;
 }
 
-// Largest b in [0, batch) with P[b] <= g (requires 0 <= g < P[batch]).
-__device__ __forceinline__ int seq_of_page(const int* P, int batch, long long g) {
-  int lo = 0, hi = batch - 1;
+// Largest v in [0, rows) with P[v] <= g (requires 0 <= g < P[rows]).
+__device__ __forceinline__ int seq_of_page(const int* P, int rows, long long g) {
+  int lo = 0, hi = rows - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if ((long long)P[mid] <= g) lo = mid; else hi = mid - 1;
@@ -120,17 +124,19 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   int* sfirst = ws_at<int>(ws, L.off_seq_first);
   int* snseg = ws_at<int>(ws, L.off_seq_nseg);
   int4* seg = ws_at<int4>(ws, L.off_seg);
-  const int batch = L.batch, n_q = L.n_q, W = L.workers;
+  const int n_q = L.n_q, W = L.workers;
+  const int rows = L.batch * n_q;  // query rows
 
-  auto pages_of = [&](int b) -> int {
+  auto pages_of = [&](int v) -> int {
+    const int b = v / n_q, j = v % n_q;
     const int len = seq_lens[b];
     if (len < n_q || len > max_blocks * bs) {
-      report(MLA_ERR_BOUNDS, 4, b, len);
+      if (j == 0) report(MLA_ERR_BOUNDS, 4, b, len);
       return 0;
     }
-    return (len + bs - 1) / bs;
+    return (len - n_q + j + 1 + bs - 1) / bs;
   };
-  const int NB = block_scan_exclusive(pages_of, P, batch);
+  const int NB = block_scan_exclusive(pages_of, P, rows);
 
   auto range_of = [&](int w, long long& s, long long& e) {
     s = (long long)w * NB / W;
@@ -140,7 +146,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
     long long s, e;
     range_of(w, s, e);
     if (s >= e) return 0;
-    return seq_of_page(P, batch, e - 1) - seq_of_page(P, batch, s) + 1;
+    return seq_of_page(P, rows, e - 1) - seq_of_page(P, rows, s) + 1;
   };
   const int nsegs = block_scan_exclusive(segs_of, wfirst, W);
 
@@ -148,7 +154,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
     long long s, e;
     range_of(w, s, e);
     if (s >= e) continue;
-    const int b0 = seq_of_page(P, batch, s), b1 = seq_of_page(P, batch, e - 1);
+    const int b0 = seq_of_page(P, rows, s), b1 = seq_of_page(P, rows, e - 1);
     int k = wfirst[w];
     for (int b = b0; b <= b1; ++b, ++k) {
       const long long lo = s > P[b] ? s : P[b];
@@ -156,7 +162,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
       seg[k] = make_int4(b, (int)(lo - P[b]), (int)(hi - P[b]), w);
     }
   }
-  for (int b = threadIdx.x; b < batch; b += blockDim.x) {
+  for (int b = threadIdx.x; b < rows; b += blockDim.x) {
     sfirst[b] = 0;
     snseg[b] = 0;
   }
@@ -173,7 +179,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   if (threadIdx.x == 0) {
     DecodeHeader* h = ws_at<DecodeHeader>(ws, 0);
     h->magic = kPlanMagic;
-    h->batch = batch;
+    h->batch = L.batch;
     h->n_q = n_q;
     h->H = L.H;
     h->d_c = L.d_c;
@@ -184,38 +190,37 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   }
 }
 
-// o_lat[t, h, :] = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M) over the
-// segments of token t's sequence.  Grid (tokens, heads), block over d_c.
+// o_lat[v, h, :] = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M) over the
+// segments of query row v.  Grid (query rows, heads), block over d_c.
 __global__ void __launch_bounds__(128) combine_kernel(const void* ws, long long ws_bytes, int batch,
                                                       int n_q, int H, int d_c, float* __restrict__ o_lat) {
   const DecodeHeader* hd = ws_at<DecodeHeader>(ws, 0);
-  const int t = blockIdx.x, h = blockIdx.y;
-  float* out = o_lat + ((long long)t * H + h) * d_c;
+  const int v = blockIdx.x, h = blockIdx.y;
+  float* out = o_lat + ((long long)v * H + h) * d_c;
   if (hd->magic != kPlanMagic || hd->batch != batch || hd->n_q != n_q || hd->H != H ||
       hd->d_c != d_c || hd->layout.total > ws_bytes) {
-    if (t == 0 && h == 0 && threadIdx.x == 0) report(MLA_ERR_WORKSPACE, 0, batch, n_q);
+    if (v == 0 && h == 0 && threadIdx.x == 0) report(MLA_ERR_WORKSPACE, 0, batch, n_q);
     for (int d = threadIdx.x; d < d_c; d += blockDim.x) out[d] = 0.f;
     return;
   }
   const DecodeLayout L = hd->layout;
-  const int b = t / n_q, j = t % n_q;
-  const int first = ws_at<int>(ws, L.off_seq_first)[b];
-  const int n = ws_at<int>(ws, L.off_seq_nseg)[b];
+  const int first = ws_at<int>(ws, L.off_seq_first)[v];
+  const int n = ws_at<int>(ws, L.off_seq_nseg)[v];
   const float* lse = ws_at<float>(ws, L.off_lse);
   const float* part = ws_at<float>(ws, L.off_o);
   float M = -INFINITY;
-  for (int s = 0; s < n; ++s) M = fmaxf(M, lse[((long long)(first + s) * n_q + j) * H + h]);
+  for (int s = 0; s < n; ++s) M = fmaxf(M, lse[(long long)(first + s) * H + h]);
   if (n == 0 || M == -INFINITY) {
     for (int d = threadIdx.x; d < d_c; d += blockDim.x) out[d] = 0.f;
     return;
   }
   float Z = 0.f;
-  for (int s = 0; s < n; ++s) Z += exp2f(lse[((long long)(first + s) * n_q + j) * H + h] - M);
+  for (int s = 0; s < n; ++s) Z += exp2f(lse[(long long)(first + s) * H + h] - M);
   const float invZ = 1.f / Z;
   for (int d = threadIdx.x; d < d_c; d += blockDim.x) {
     float acc = 0.f;
     for (int s = 0; s < n; ++s) {
-      const long long r = ((long long)(first + s) * n_q + j) * H + h;
+      const long long r = (long long)(first + s) * H + h;
       acc += exp2f(lse[r] - M) * part[r * d_c + d];
     }
     out[d] = acc * invZ;

@@ -1,7 +1,7 @@
-// Latent-space decode on CUDA cores: one warp per (segment, query, head).
+// Latent-space decode on CUDA cores: one warp per (segment, head).
 // Used for the fp32 storage path (small shapes, exact fp32 arithmetic).
 //
-// For its rows u of the segment (u <= the query's position p):
+// For the rows u of its segment (all visible to the segment's query row):
 //   s_u = (q_lat . c_u + q_R . kR_u) * scale * log2(e)
 // with an online (running-max) softmax, O = sum_u 2^(s_u - m) c_u / l.
 #pragma once
@@ -14,7 +14,7 @@ constexpr int kSimtDecodeMaxRow = 1024;  // d_c + d_r handled by one warp (32 la
 
 template <typename T, int DPL>
 __global__ void __launch_bounds__(128) decode_simt_kernel(
-    const T* __restrict__ q_lat, const T* __restrict__ q_rope, const T* __restrict__ pool,
+    const float* __restrict__ q_lat, const float* __restrict__ q_rope, const T* __restrict__ pool,
     const int32_t* __restrict__ block_table, int max_blocks, int num_blocks,
     const int32_t* __restrict__ seq_lens, int n_q, int H, int d_c, int d_r, int bs,
     float scale_log2, void* ws, DecodeLayout L) {
@@ -22,29 +22,26 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(
   const int sidx = blockIdx.x;
   if (sidx >= hd->num_segments) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int idx = blockIdx.y * 4 + warp;
-  if (idx >= n_q * H) return;
-  const int j = idx / H, h = idx % H;
+  const int h = blockIdx.y * 4 + warp;
+  if (h >= H) return;
   const int4 sg = ws_at<int4>(ws, L.off_seg)[sidx];
-  const int b = sg.x;
-  const int t = b * n_q + j;
-  const int p = seq_lens[b] - n_q + j;  // last row this query sees
+  const int v = sg.x, b = v / n_q, j = v % n_q;
+  const int len_v = seq_lens[b] - n_q + j + 1;  // rows this query sees
   const int row = d_c + d_r;
 
   float q[DPL], o[DPL];
 #pragma unroll
   for (int i = 0; i < DPL; ++i) {
     const int d = lane + 32 * i;
-    float v = 0.f;
-    if (d < d_c) v = Store<T>::ld(q_lat + ((long long)t * H + h) * d_c + d);
-    else if (d < row) v = Store<T>::ld(q_rope + ((long long)t * H + h) * d_r + (d - d_c));
-    q[i] = v;
+    float val = 0.f;
+    if (d < d_c) val = q_lat[((long long)v * H + h) * d_c + d];
+    else if (d < row) val = q_rope[((long long)v * H + h) * d_r + (d - d_c)];
+    q[i] = val;
     o[i] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
   for (int blk = sg.y; blk < sg.z; ++blk) {
-    const int u0 = blk * bs;
-    const int nrows = min(bs, p + 1 - u0);
+    const int nrows = min(bs, len_v - blk * bs);
     if (nrows <= 0) break;
     const int phys = block_table[(long long)b * max_blocks + blk];
     if (phys < 0 || phys >= num_blocks) {
@@ -75,7 +72,7 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(
       m = m_new;
     }
   }
-  const long long r_out = ((long long)sidx * n_q + j) * H + h;
+  const long long r_out = (long long)sidx * H + h;
   const float inv = l > 0.f ? 1.f / l : 0.f;
   float* out = ws_at<float>(ws, L.off_o) + r_out * d_c;
 #pragma unroll

@@ -21,6 +21,7 @@ mla_status check_cfg(const mla_config* c) {
       !(c->rope_theta > 0.0) || c->softmax_scale < 0.f)
     return MLA_ERR_INVALID_ARG;
   if (c->dtype != MLA_F32 && c->dtype != MLA_BF16) return MLA_ERR_INVALID_ARG;
+  if (c->flags & ~MLA_FLAG_SPLIT_QUERY) return MLA_ERR_INVALID_ARG;
   return MLA_OK;
 }
 
@@ -58,8 +59,8 @@ mla_status append_impl(const mla_config* c, const void* x, int n, const void* W_
                        cudaStream_t s) {
   const int row = c->d_c + c->d_r;
   double* C = static_cast<double*>(ws);
-  MLA_CUDA((gemm_rm<T, double>(x, c->hidden, W_DKV, c->d_c, C, row, n, c->d_c, c->hidden, s)));
-  MLA_CUDA((gemm_rm<T, double>(x, c->hidden, W_KR, c->d_r, C + c->d_c, row, n, c->d_r, c->hidden, s)));
+  MLA_CUDA((gemm_rm<T, T, double>(x, c->hidden, W_DKV, c->d_c, C, row, n, c->d_c, c->hidden, s)));
+  MLA_CUDA((gemm_rm<T, T, double>(x, c->hidden, W_KR, c->d_r, C + c->d_c, row, n, c->d_r, c->hidden, s)));
   const long long total = (long long)n * (c->d_c + c->d_r / 2);
   append_finish_kernel<T><<<grid_for(total), 256, 0, s>>>(
       C, n, c->d_c, c->d_r, c->rope_theta, seq_idx, pos, static_cast<T*>(k->pool), k->block_table,
@@ -69,68 +70,61 @@ mla_status append_impl(const mla_config* c, const void* x, int n, const void* W_
 }
 
 // ---------------------------------------------------------------- absorb
+// Query intermediates stay in fp32: with bf16 weights and fp32 activations the
+// only rounding left on the query side is fp32 accumulation.
 struct AbsorbWs {
-  size_t cq_f, cq_t, q_f, qn_t, ql_f, total;
+  size_t cq_f, q_f, qn_f, total;
 };
 AbsorbWs absorb_ws(const mla_config* c, int n) {
-  const size_t eb = elem_bytes(c);
   const size_t H = c->n_heads, qw = H * (c->qk_nope + c->d_r);
   AbsorbWs w{};
   size_t o = 0;
   w.cq_f = o; o = align_up(o + 4 * (size_t)n * c->q_lora, 256);
-  w.cq_t = o; o = align_up(o + eb * (size_t)n * c->q_lora, 256);
   w.q_f = o;  o = align_up(o + 4 * (size_t)n * qw, 256);
-  w.qn_t = o; o = align_up(o + eb * (size_t)n * H * c->qk_nope, 256);
-  w.ql_f = o; o = align_up(o + 4 * (size_t)n * H * c->d_c, 256);
+  w.qn_f = o; o = align_up(o + 4 * (size_t)n * H * c->qk_nope, 256);
   w.total = o;
   return w;
 }
 
 template <typename T>
 mla_status absorb_impl(const mla_config* c, const void* x, int n, const void* W_DQ, const void* W_UQ,
-                       const void* W_UK, const int32_t* pos, void* q_lat, void* q_rope, void* ws,
+                       const void* W_UK, const int32_t* pos, float* q_lat, float* q_rope, void* ws,
                        cudaStream_t s) {
   const AbsorbWs w = absorb_ws(c, n);
   char* base = static_cast<char*>(ws);
   float* cq_f = reinterpret_cast<float*>(base + w.cq_f);
-  T* cq_t = reinterpret_cast<T*>(base + w.cq_t);
   float* q_f = reinterpret_cast<float*>(base + w.q_f);
-  T* qn_t = reinterpret_cast<T*>(base + w.qn_t);
-  float* ql_f = reinterpret_cast<float*>(base + w.ql_f);
+  float* qn_f = reinterpret_cast<float*>(base + w.qn_f);
   const int H = c->n_heads, nope = c->qk_nope, qw = H * (nope + c->d_r);
   if (c->q_lora > 0) {
-    MLA_CUDA((gemm_rm<T, float>(x, c->hidden, W_DQ, c->q_lora, cq_f, c->q_lora, n, c->q_lora, c->hidden, s)));
-    MLA_CUDA(round_store<T>(cq_f, cq_t, (long long)n * c->q_lora, s));
-    MLA_CUDA((gemm_rm<T, float>(cq_t, c->q_lora, W_UQ, qw, q_f, qw, n, qw, c->q_lora, s)));
+    MLA_CUDA((gemm_rm<T, T, float>(x, c->hidden, W_DQ, c->q_lora, cq_f, c->q_lora, n, c->q_lora, c->hidden, s)));
+    MLA_CUDA((gemm_rm<float, T, float>(cq_f, c->q_lora, W_UQ, qw, q_f, qw, n, qw, c->q_lora, s)));
   } else {
-    MLA_CUDA((gemm_rm<T, float>(x, c->hidden, W_UQ, qw, q_f, qw, n, qw, c->hidden, s)));
+    MLA_CUDA((gemm_rm<T, T, float>(x, c->hidden, W_UQ, qw, q_f, qw, n, qw, c->hidden, s)));
   }
   const long long tot = (long long)n * H * (nope + c->d_r / 2);
-  query_split_kernel<T><<<grid_for(tot), 256, 0, s>>>(q_f, n, H, nope, c->d_r, c->rope_theta, pos, qn_t,
-                                                      static_cast<T*>(q_rope));
+  query_split_kernel<float><<<grid_for(tot), 256, 0, s>>>(q_f, n, H, nope, c->d_r, c->rope_theta, pos,
+                                                          qn_f, q_rope);
   note_launch();
   MLA_CUDA(cudaGetLastError());
   // q_lat[t, h, :] = q_nope[t, h, :] W_UK_h^T, batched over heads
-  GemmSimtArgs g{qn_t, W_UK, ql_f, n, c->d_c, nope, H,
+  GemmSimtArgs g{qn_f, W_UK, q_lat, n, c->d_c, nope, H,
                  (long long)H * nope, 1, nope,
                  1, (long long)H * nope, nope,
                  (long long)H * c->d_c, 1, c->d_c};
-  MLA_CUDA((gemm_simt<T, float>(g, s)));
-  MLA_CUDA(round_store<T>(ql_f, static_cast<T*>(q_lat), (long long)n * H * c->d_c, s));
+  MLA_CUDA((gemm_simt<float, T, float>(g, s)));
   return MLA_OK;
 }
 
 // ---------------------------------------------------------------- out proj
 struct OutWs {
-  size_t ol_t, oh_f, oh_t, y_f, total;
+  size_t oh_f, y_f, total;
 };
 OutWs out_ws(const mla_config* c, int n) {
-  const size_t eb = elem_bytes(c), H = c->n_heads;
+  const size_t H = c->n_heads;
   OutWs w{};
   size_t o = 0;
-  w.ol_t = o; o = align_up(o + eb * (size_t)n * H * c->d_c, 256);
   w.oh_f = o; o = align_up(o + 4 * (size_t)n * H * c->v_head, 256);
-  w.oh_t = o; o = align_up(o + eb * (size_t)n * H * c->v_head, 256);
   w.y_f = o;  o = align_up(o + 4 * (size_t)n * c->hidden, 256);
   w.total = o;
   return w;
@@ -141,20 +135,16 @@ mla_status out_impl(const mla_config* c, const float* o_lat, int n, const void* 
                     void* y, void* ws, cudaStream_t s) {
   const OutWs w = out_ws(c, n);
   char* base = static_cast<char*>(ws);
-  T* ol_t = reinterpret_cast<T*>(base + w.ol_t);
   float* oh_f = reinterpret_cast<float*>(base + w.oh_f);
-  T* oh_t = reinterpret_cast<T*>(base + w.oh_t);
   float* y_f = reinterpret_cast<float*>(base + w.y_f);
   const int H = c->n_heads, dv = c->v_head;
-  MLA_CUDA(round_store<T>(o_lat, ol_t, (long long)n * H * c->d_c, s));
   // o_h[t, h, :] = o_lat[t, h, :] W_UV_h, batched over heads
-  GemmSimtArgs g{ol_t, W_UV, oh_f, n, dv, c->d_c, H,
+  GemmSimtArgs g{o_lat, W_UV, oh_f, n, dv, c->d_c, H,
                  (long long)H * c->d_c, 1, c->d_c,
                  (long long)H * dv, 1, dv,
                  (long long)H * dv, 1, dv};
-  MLA_CUDA((gemm_simt<T, float>(g, s)));
-  MLA_CUDA(round_store<T>(oh_f, oh_t, (long long)n * H * dv, s));
-  MLA_CUDA((gemm_rm<T, float>(oh_t, (long long)H * dv, W_O, c->hidden, y_f, c->hidden, n, c->hidden, H * dv, s)));
+  MLA_CUDA((gemm_simt<float, T, float>(g, s)));
+  MLA_CUDA((gemm_rm<float, T, float>(oh_f, (long long)H * dv, W_O, c->hidden, y_f, c->hidden, n, c->hidden, H * dv, s)));
   MLA_CUDA(round_store<T>(y_f, static_cast<T*>(y), (long long)n * c->hidden, s));
   return MLA_OK;
 }
@@ -170,20 +160,20 @@ int resolve_workers(const mla_config* c, int max_workers) {
 }
 
 template <typename T, int DPL>
-void launch_decode_simt(const mla_config* c, const void* q_lat, const void* q_rope, int n_q,
+void launch_decode_simt(const mla_config* c, const float* q_lat, const float* q_rope, int n_q,
                         const mla_cache* k, const int32_t* seq_lens, void* ws, const DecodeLayout& L,
                         cudaStream_t s) {
   const float scale_log2 = scale_of(c) * 1.4426950408889634f;
-  dim3 grid(L.max_segments, (n_q * c->n_heads + 3) / 4);
+  dim3 grid(L.max_segments, (c->n_heads + 3) / 4);
   decode_simt_kernel<T, DPL><<<grid, 128, 0, s>>>(
-      static_cast<const T*>(q_lat), static_cast<const T*>(q_rope), static_cast<const T*>(k->pool),
+      q_lat, q_rope, static_cast<const T*>(k->pool),
       k->block_table, k->max_blocks_per_seq, k->num_blocks, seq_lens, n_q, c->n_heads, c->d_c, c->d_r,
       c->block_size, scale_log2, ws, L);
   note_launch();
 }
 
 template <typename T>
-mla_status decode_simt_dispatch(const mla_config* c, const void* q_lat, const void* q_rope, int n_q,
+mla_status decode_simt_dispatch(const mla_config* c, const float* q_lat, const float* q_rope, int n_q,
                                 const mla_cache* k, const int32_t* seq_lens, void* ws,
                                 const DecodeLayout& L, cudaStream_t s) {
   const int row = c->d_c + c->d_r;
@@ -241,8 +231,8 @@ size_t mla_absorb_q_workspace_size(const mla_config* cfg, int32_t n_tok) {
 }
 
 mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok, const void* W_DQ,
-                        const void* W_UQ, const void* W_UK, const int32_t* pos, void* q_lat,
-                        void* q_rope, void* workspace, size_t ws_bytes, void* stream) {
+                        const void* W_UQ, const void* W_UK, const int32_t* pos, float* q_lat,
+                        float* q_rope, void* workspace, size_t ws_bytes, void* stream) {
   MLA_TRY(check_cfg(cfg));
   if (n_tok < 0) return MLA_ERR_INVALID_ARG;
   if (n_tok == 0) return MLA_OK;
@@ -260,7 +250,7 @@ size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t n
   return (size_t)decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers)).total;
 }
 
-mla_status mla_decode(const mla_config* cfg, const void* q_lat, const void* q_rope, int32_t batch,
+mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_rope, int32_t batch,
                       int32_t n_q, const mla_cache* cache, const int32_t* seq_lens, int32_t max_workers,
                       void* workspace, size_t ws_bytes, void* stream) {
   MLA_TRY(check_cfg(cfg));

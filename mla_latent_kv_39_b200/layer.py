@@ -25,8 +25,8 @@ class DecodeLayer:
         dev = cache.pool.device
         dt = cfg.torch_dtype
         H = cfg.n_heads
-        self.q_lat = torch.empty(n, H, cfg.d_c, dtype=dt, device=dev)
-        self.q_rope = torch.empty(n, H, cfg.d_r, dtype=dt, device=dev)
+        self.q_lat = torch.empty(n, H, cfg.d_c, dtype=torch.float32, device=dev)
+        self.q_rope = torch.empty(n, H, cfg.d_r, dtype=torch.float32, device=dev)
         self.o_lat = torch.empty(n, H, cfg.d_c, dtype=torch.float32, device=dev)
         self.y = torch.empty(n, cfg.hidden, dtype=dt, device=dev)
         gemm_ws = max(abi.mla_cache_append_workspace_size(cfg, n), abi.mla_absorb_q_workspace_size(cfg, n),
@@ -35,7 +35,15 @@ class DecodeLayer:
         self.ws_decode = torch.empty(abi.mla_decode_workspace_size(cfg, batch, n_q, max_workers),
                                      dtype=torch.uint8, device=dev)
 
+    def _gemm_ws(self, n: int) -> torch.Tensor:
+        need = max(abi.mla_cache_append_workspace_size(self.cfg, n), abi.mla_absorb_q_workspace_size(self.cfg, n),
+                   abi.mla_out_proj_workspace_size(self.cfg, n))
+        if need > self.ws_gemm.numel():
+            self.ws_gemm = torch.empty(need, dtype=torch.uint8, device=self.ws_gemm.device)
+        return self.ws_gemm
+
     def append(self, x, seq_idx, pos, stream=None):
+        self._gemm_ws(x.shape[0])
         abi.mla_cache_append(self.cfg, x, self.W["W_DKV"], self.W["W_KR"], seq_idx, pos, self.cache,
                              self.ws_gemm, stream)
 

@@ -96,12 +96,19 @@ def test_physical_page_order_does_not_change_the_result():
 
 def test_bad_block_id_is_reported_not_faulted():
     wl = reduced(WORKLOADS["v3_b64_ragged1k_8k"], lengths=[200, 100])
-    data = generate(wl)
-    data.block_table[1, 0] = data.num_blocks + 5      # outside the pool
-    with pytest.raises(MLAError) as e:
-        run_gpu(wl, data=data)
-    assert e.value.status == abi.MLA_ERR_BOUNDS
+    data, dev, layer = run_gpu(wl)
+    dev["block_table"][1, 0] = data.num_blocks + 5      # outside the pool
+    layer.decode(dev["seq_lens"])
+    status, detail = mla_get_device_error()
+    assert status == abi.MLA_ERR_BOUNDS and detail[1] == 1
     assert mla_get_device_error()[0] == abi.MLA_OK    # cleared by the first read
+    dev["block_table"][1, 0] = 0
+    pos = torch.tensor([130], dtype=torch.int32, device="cuda")
+    seq = torch.tensor([1], dtype=torch.int32, device="cuda")
+    dev["block_table"][1, 2] = -7                        # append into a missing page
+    layer.append(dev["x_new"][1:2], seq, pos)
+    status, detail = mla_get_device_error()
+    assert status == abi.MLA_ERR_BOUNDS
 
 
 def test_sequence_shorter_than_its_queries_is_reported():
@@ -141,8 +148,8 @@ def test_empty_batch_is_a_no_op():
     _, dev, layer = run_gpu(wl)
     cfg = layer.cfg
     H = cfg.n_heads
-    e = torch.empty(0, H, cfg.d_c, dtype=torch.bfloat16, device="cuda")
-    abi.mla_decode(cfg, e, torch.empty(0, H, cfg.d_r, dtype=torch.bfloat16, device="cuda"), 0, 1,
+    e = torch.empty(0, H, cfg.d_c, dtype=torch.float32, device="cuda")
+    abi.mla_decode(cfg, e, torch.empty(0, H, cfg.d_r, dtype=torch.float32, device="cuda"), 0, 1,
                    layer.cache, torch.empty(0, dtype=torch.int32, device="cuda"), layer.ws_decode, 0)
     torch.cuda.synchronize()
     check_device_error()
