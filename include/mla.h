@@ -124,6 +124,35 @@ mla_status mla_cache_append(const mla_config* cfg, const void* x, int32_t n_tok,
                             void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Latent append for callers that cannot allocate device memory.  The pages
+ * have no counterpart for this entry point; it exists for callers such as a
+ * serving engine that has already reserved all device memory for its own
+ * pool and forbids any further cudaMalloc, or plain C callers without a
+ * device allocator, which cannot provide the workspace mla_cache_append
+ * asks for.
+ * Same arguments and result as mla_cache_append, minus the workspace: its
+ * scratch is a fixed array of MLA_APPEND_NOALLOC_SCRATCH_BYTES in device
+ * memory, built into the library, which every GPU that loads the library
+ * holds until the process exits.  The call allocates nothing and frees
+ * nothing.  The caller still passes all inputs and outputs.
+ *  - Size limit: n_tok must satisfy
+ *      mla_cache_append_workspace_size(cfg, n_tok) <= MLA_APPEND_NOALLOC_SCRATCH_BYTES
+ *    (n_tok <= 910 for d_c + d_r = 576); larger requests return
+ *    MLA_ERR_WORKSPACE before any launch.
+ *  - First call on a device: it looks up the device address of the array
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make
+ *    that first call before any stream capture on that device.
+ *  - All calls on a device share the one array.  Calls that may overlap on
+ *    the GPU (different streams, no ordering between them) race on it and
+ *    corrupt each other's result; serialise them, e.g. on one stream.
+ * ------------------------------------------------------------------------- */
+#define MLA_APPEND_NOALLOC_SCRATCH_BYTES (4u << 20)
+mla_status mla_cache_append_noalloc(const mla_config* cfg, const void* x, int32_t n_tok,
+                                    const void* W_DKV, const void* W_KR,
+                                    const int32_t* seq_idx, const int32_t* pos,
+                                    const mla_cache* cache, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Step 2 - queries with W_UK absorbed ([P2] query compression; [P5] section 1
  * "Định nghĩa": the decompression matrix is folded into the query matrix, the
  * RoPE part stays separate).

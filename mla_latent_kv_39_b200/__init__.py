@@ -15,6 +15,7 @@ from .abi import (  # noqa: F401
     mla_absorb_q_workspace_size,
     mla_cache_append,
     mla_cache_append_workspace_size,
+    mla_cache_append_noalloc,
     mla_combine,
     mla_decode,
     mla_decode_workspace_size,

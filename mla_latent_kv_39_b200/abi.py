@@ -29,6 +29,7 @@ MLA_ERR_WORKSPACE = -6
 MLA_F32 = 0
 MLA_BF16 = 1
 MLA_FLAG_SPLIT_QUERY = 1
+MLA_APPEND_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 # Every symbol the header declares, with (restype, argtypes).
 _vp, _i32, _sz, _d, _f = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_double, ctypes.c_float
@@ -59,6 +60,7 @@ SIGNATURES = {
     "mla_status_string": (ctypes.c_char_p, [_i32]),
     "mla_cache_append_workspace_size": (_sz, [_P_CFG, _i32]),
     "mla_cache_append": (_i32, [_P_CFG, _vp, _i32, _vp, _vp, _vp, _vp, _P_CACHE, _vp, _sz, _vp]),
+    "mla_cache_append_noalloc": (_i32, [_P_CFG, _vp, _i32, _vp, _vp, _vp, _vp, _P_CACHE, _vp]),
     "mla_absorb_q_workspace_size": (_sz, [_P_CFG, _i32]),
     "mla_absorb_q": (_i32, [_P_CFG, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mla_decode_workspace_size": (_sz, [_P_CFG, _i32, _i32, _i32]),
@@ -209,6 +211,24 @@ def mla_cache_append(cfg: Config, x, W_DKV, W_KR, seq_idx, pos, cache: Cache, wo
     _check(lib().mla_cache_append(ctypes.byref(cfg.c()), _ptr(x), n, _ptr(W_DKV), _ptr(W_KR),
                                   _ptr(seq_idx), _ptr(pos), ctypes.byref(cache.c), _ptr(workspace),
                                   workspace.numel(), _stream(stream)), "mla_cache_append")
+
+
+def mla_cache_append_noalloc(cfg: Config, x, W_DKV, W_KR, seq_idx, pos, cache: Cache, stream=None):
+    """mla_cache_append without a caller workspace, for callers that cannot
+    allocate device memory: the scratch is the library's fixed device array
+    (shared by all calls on a device; overlapping calls race)."""
+    dt = cfg.torch_dtype
+    n = x.shape[0]
+    _need(x, "x", dt, shape=(n, cfg.hidden))
+    _need(W_DKV, "W_DKV", dt, shape=(cfg.hidden, cfg.d_c))
+    _need(W_KR, "W_KR", dt, shape=(cfg.hidden, cfg.d_r))
+    _need(seq_idx, "seq_idx", torch.int32, shape=(n,))
+    _need(pos, "pos", torch.int32, shape=(n,))
+    if cache.pool.dtype != dt or cache.pool.shape[1:] != (cfg.block_size, cfg.d_c + cfg.d_r):
+        raise ValueError("cache pool dtype/shape does not match the config")
+    _check(lib().mla_cache_append_noalloc(ctypes.byref(cfg.c()), _ptr(x), n, _ptr(W_DKV), _ptr(W_KR),
+                                          _ptr(seq_idx), _ptr(pos), ctypes.byref(cache.c),
+                                          _stream(stream)), "mla_cache_append_noalloc")
 
 
 def mla_absorb_q(cfg: Config, x, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, workspace, stream=None):

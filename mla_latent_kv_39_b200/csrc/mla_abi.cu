@@ -2,7 +2,9 @@
 // Every step of the path runs in the kernels included below; this file only
 // checks arguments, computes workspace offsets and launches.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
+#include <mutex>
 
 #include "common.cuh"
 #include "decode_plan.cuh"
@@ -184,6 +186,36 @@ mla_status decode_simt_dispatch(const mla_config* c, const float* q_lat, const f
   return st(cudaGetLastError());
 }
 
+// ------------------------------------------------- append without allocation
+// Scratch of mla_cache_append_noalloc: a fixed device array that every GPU
+// loading the library holds until the process exits.  In host code the name
+// g_append_scratch is only a host-side stand-in for the device symbol, never a
+// usable device address: the address comes from cudaGetSymbolAddress, taken
+// once per device (with that device current) and cached below.
+static __device__ __align__(256) unsigned char g_append_scratch[MLA_APPEND_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 128;
+std::atomic<void*> g_append_scratch_addr[kMaxDevices];
+std::mutex g_append_scratch_mutex;
+
+// Device address of this device's scratch array, looked up on first use.
+mla_status append_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  void* p = g_append_scratch_addr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> lock(g_append_scratch_mutex);
+    p = g_append_scratch_addr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+      if (cudaGetSymbolAddress(&p, g_append_scratch) != cudaSuccess || p == nullptr) return MLA_ERR_CUDA;
+      g_append_scratch_addr[dev].store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
+  return MLA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -223,6 +255,26 @@ mla_status mla_cache_append(const mla_config* cfg, const void* x, int32_t n_tok,
   if (cfg->dtype == MLA_BF16)
     return append_impl<bf16>(cfg, x, n_tok, W_DKV, W_KR, seq_idx, pos, cache, workspace, s);
   return append_impl<float>(cfg, x, n_tok, W_DKV, W_KR, seq_idx, pos, cache, workspace, s);
+}
+
+mla_status mla_cache_append_noalloc(const mla_config* cfg, const void* x, int32_t n_tok, const void* W_DKV,
+                                    const void* W_KR, const int32_t* seq_idx, const int32_t* pos,
+                                    const mla_cache* cache, void* stream) {
+  MLA_TRY(check_cfg(cfg));
+  if (n_tok < 0) return MLA_ERR_INVALID_ARG;
+  if (n_tok == 0) return MLA_OK;
+  if (!x || !W_DKV || !W_KR || !seq_idx || !pos) return MLA_ERR_INVALID_ARG;
+  MLA_TRY(check_cache(cache));
+  const size_t need = append_ws(cfg, n_tok);
+  if (need > (size_t)MLA_APPEND_NOALLOC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  MLA_TRY(append_scratch_address(&scratch));
+  // Every value of the scratch that the append reads is written first by the
+  // same call, so nothing left over from an earlier call needs clearing.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cfg->dtype == MLA_BF16)
+    return append_impl<bf16>(cfg, x, n_tok, W_DKV, W_KR, seq_idx, pos, cache, scratch, s);
+  return append_impl<float>(cfg, x, n_tok, W_DKV, W_KR, seq_idx, pos, cache, scratch, s);
 }
 
 size_t mla_absorb_q_workspace_size(const mla_config* cfg, int32_t n_tok) {
