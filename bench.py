@@ -238,7 +238,7 @@ def run_ours(args):
     wl = dataclasses.replace(base, seed=rank_seed(base.seed, rank))
     data = generate(wl)
     dev = device_inputs(data, device)
-    cfg = mla.Config.from_shape(wl.shape)
+    cfg = mla.Config.from_shape(wl.shape, split_query=wl.split_query)
     cache = mla.Cache(dev["pool"], dev["block_table"])
     layer = mla.DecodeLayer(cfg, dev["weights"], cache, wl.batch, wl.n_q, args.max_workers)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)

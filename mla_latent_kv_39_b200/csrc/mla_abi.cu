@@ -9,6 +9,7 @@
 #include "common.cuh"
 #include "decode_plan.cuh"
 #include "decode_simt.cuh"
+#include "decode_tc.cuh"
 #include "elementwise.cuh"
 #include "gemm_simt.cuh"
 
@@ -152,9 +153,12 @@ mla_status out_impl(const mla_config* c, const float* o_lat, int n, const void* 
 }
 
 // ---------------------------------------------------------------- decode
+// Parallel workers of the decode: one CTA pair per two SMs on the
+// tensor-core path (bf16), two warps-worth of CTAs per SM on the CUDA-core path.
 int default_workers(const mla_config* c) {
-  const int sms = device_sm_count();
-  return std::max(1, 2 * (sms > 0 ? sms : 148));
+  const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+  if (c->dtype == MLA_BF16) return std::max(1, sms / 2);
+  return std::max(1, 2 * sms);
 }
 
 int resolve_workers(const mla_config* c, int max_workers) {
@@ -311,6 +315,7 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
   if (!q_lat || !q_rope || !seq_lens || !workspace) return MLA_ERR_INVALID_ARG;
   MLA_TRY(check_cache(cache));
   if (cache->batch < batch) return MLA_ERR_INVALID_ARG;
+  if (cfg->dtype == MLA_BF16 && !tcdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
   const DecodeLayout L =
       decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers));
   if (ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
@@ -319,7 +324,7 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
   note_launch();
   MLA_CUDA(cudaGetLastError());
   if (cfg->dtype == MLA_BF16)
-    return decode_simt_dispatch<bf16>(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, s);
+    return tcdec::launch(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, scale_of(cfg), s);
   return decode_simt_dispatch<float>(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, s);
 }
 

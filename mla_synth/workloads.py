@@ -111,6 +111,9 @@ class Workload:
     spike_scale: float = 1.0
     seed: int = 0
     description: str = ""
+    # run option, not data: hold the query as a bf16 hi + lo pair in the decode
+    # (strongly peaked softmaxes need more than bf16's 8 significant bits)
+    split_query: bool = False
 
     @property
     def n_tok(self) -> int:
@@ -132,7 +135,7 @@ WORKLOADS: Dict[str, Workload] = {
                     "64-token pages in shuffled order"),
     "v3_b4_long": Workload(
         "v3_b4_long", SHAPES["v3"], batch=4, n_q=1, lengths=(65536, 131072, 32768, 100000),
-        spike_frac=0.01, spike_scale=8.0,
+        spike_frac=0.01, spike_scale=8.0, split_query=True,
         description="V3-shaped long-context split-KV stress, contexts 65536/131072/32768/100000, "
                     "1% of latent rows scaled x8"),
     "v3_b128_nq2_ragged512_16k": Workload(

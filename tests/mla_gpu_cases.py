@@ -21,7 +21,7 @@ def tol_for(shape) -> float:
 def run_gpu(wl, data=None, max_workers: int = 0, pool: Optional[torch.Tensor] = None):
     data = data if data is not None else generate(wl)
     dev = device_inputs(data, "cuda", pool=pool)
-    cfg = Config.from_shape(wl.shape)
+    cfg = Config.from_shape(wl.shape, split_query=wl.split_query)
     cache = Cache(dev["pool"], dev["block_table"])
     layer = DecodeLayer(cfg, dev["weights"], cache, wl.batch, wl.n_q, max_workers)
     if wl.cached_from_append:
