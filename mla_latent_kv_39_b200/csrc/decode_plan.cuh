@@ -116,10 +116,14 @@ __device__ __forceinline__ int seq_of_page(const int* P, int rows, long long g) 
   return lo;
 }
 
+// Page prefix of the query rows lives in shared memory (the searches below
+// are chains of dependent loads); one CTA computes the whole plan.
+constexpr int kPlanMaxRows = 49152;
+
 __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __restrict__ seq_lens,
                                                            int bs, int max_blocks, void* ws,
                                                            DecodeLayout L) {
-  int* P = ws_at<int>(ws, L.off_prefix);
+  extern __shared__ int P[];  // [rows + 1]
   int* wfirst = ws_at<int>(ws, L.off_worker_first);
   int* sfirst = ws_at<int>(ws, L.off_seq_first);
   int* snseg = ws_at<int>(ws, L.off_seq_nseg);

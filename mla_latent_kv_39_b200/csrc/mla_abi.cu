@@ -313,6 +313,7 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
   if (batch < 0 || n_q <= 0 || max_workers < 0) return MLA_ERR_INVALID_ARG;
   if (batch == 0) return MLA_OK;
   if (!q_lat || !q_rope || !seq_lens || !workspace) return MLA_ERR_INVALID_ARG;
+  if ((long long)batch * n_q > kPlanMaxRows) return MLA_ERR_UNSUPPORTED;
   MLA_TRY(check_cache(cache));
   if (cache->batch < batch) return MLA_ERR_INVALID_ARG;
   if (cfg->dtype == MLA_BF16 && !tcdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
@@ -320,7 +321,12 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
       decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers));
   if (ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  decode_plan_kernel<<<1, 1024, 0, s>>>(seq_lens, cfg->block_size, cache->max_blocks_per_seq, workspace, L);
+  const size_t plan_smem = sizeof(int) * ((size_t)batch * n_q + 1);
+  if (plan_smem > 48 * 1024 &&
+      cudaFuncSetAttribute(decode_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan_smem) !=
+          cudaSuccess)
+    return MLA_ERR_CUDA;
+  decode_plan_kernel<<<1, 1024, plan_smem, s>>>(seq_lens, cfg->block_size, cache->max_blocks_per_seq, workspace, L);
   note_launch();
   MLA_CUDA(cudaGetLastError());
   if (cfg->dtype == MLA_BF16)
