@@ -113,7 +113,7 @@ class ClockSampler:
     def _handle(self):
         import pynvml
         pynvml.nvmlInit()
-        u = torch.cuda.get_device_properties(self.index).uuid.bytes.hex()
+        u = bytes(torch.cuda.get_device_properties(self.index).uuid.bytes).hex()
         uuid = f"GPU-{u[0:8]}-{u[8:12]}-{u[12:16]}-{u[16:20]}-{u[20:32]}"
         return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid)
 

@@ -45,11 +45,12 @@ __device__ __forceinline__ long long cache_row_slot(const int32_t* seq_idx, cons
   return (long long)phys * bs + (p % bs);
 }
 
-// New latent rows from exact (fp64) projections C = x [W_DKV | W_KR]:
+// New latent rows from exact (fp64) projections C = x [W_DKV | W_KR] (the sum
+// of `splits` fp64 partials over K):
 // c = C[:, :d_c], k_R = RoPE(C[:, d_c:], pos); each value rounded once to T
 // and written to its paged slot.  One thread per latent value or rotary pair.
 template <typename T>
-__global__ void append_finish_kernel(const double* __restrict__ C, int n_tok, int d_c, int d_r,
+__global__ void append_finish_kernel(const double* __restrict__ C, int splits, int n_tok, int d_c, int d_r,
                                      double theta, const int32_t* __restrict__ seq_idx,
                                      const int32_t* __restrict__ pos, T* __restrict__ pool,
                                      const int32_t* __restrict__ block_table, int batch,
@@ -62,16 +63,22 @@ __global__ void append_finish_kernel(const double* __restrict__ C, int n_tok, in
     const long long slot = cache_row_slot(seq_idx, pos, t, block_table, batch, max_blocks, num_blocks, bs);
     if (slot < 0) continue;
     const int row = d_c + d_r;
+    const long long split_stride = (long long)n_tok * row;
     const double* src = C + (long long)t * row;
+    auto total = [&](int col) {
+      double acc = 0.0;
+      for (int s = 0; s < splits; ++s) acc += src[s * split_stride + col];
+      return acc;
+    };
     T* dst = pool + slot * row;
     if (k < d_c) {
-      Store<T>::st64(dst + k, src[k]);
+      Store<T>::st64(dst + k, total(k));
     } else {
       const int pr = k - d_c;  // rotary pair index
       const double ang = (double)pos[t] * rope_inv_freq(theta, pr, d_r);
       double sn, cs;
       sincos(ang, &sn, &cs);
-      const double r0 = src[d_c + 2 * pr], r1 = src[d_c + 2 * pr + 1];
+      const double r0 = total(d_c + 2 * pr), r1 = total(d_c + 2 * pr + 1);
       Store<T>::st64(dst + d_c + 2 * pr, r0 * cs - r1 * sn);
       Store<T>::st64(dst + d_c + 2 * pr + 1, r0 * sn + r1 * cs);
     }
@@ -103,6 +110,37 @@ __global__ void query_split_kernel(const float* __restrict__ q, int n_tok, int H
       const double r0 = src[nope + 2 * pr], r1 = src[nope + 2 * pr + 1];
       Store<T>::st(q_rope + th * d_r + 2 * pr, (float)(r0 * cs - r1 * sn));
       Store<T>::st(q_rope + th * d_r + 2 * pr + 1, (float)(r0 * sn + r1 * cs));
+    }
+  }
+}
+
+// Split q [n, H, nope + d_r] (fp32): q_nope to bf16 (and its bf16 remainder
+// when lo != nullptr), the rotated q_rope kept in fp32 (angle and rotation in fp64).
+__global__ void query_split_bf16_kernel(const float* __restrict__ q, int n_tok, int H, int nope, int d_r,
+                                        double theta, const int32_t* __restrict__ pos, bf16* __restrict__ q_nope,
+                                        bf16* __restrict__ q_nope_lo, float* __restrict__ q_rope) {
+  const int w = nope + d_r;
+  const int per_head = nope + d_r / 2;
+  const long long total = (long long)n_tok * H * per_head;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long th = i / per_head;
+    const int k = (int)(i % per_head);
+    const int t = (int)(th / H);
+    const float* src = q + th * w;
+    if (k < nope) {
+      const float v = src[k];
+      const bf16 h = __float2bfloat16_rn(v);
+      q_nope[th * nope + k] = h;
+      if (q_nope_lo) q_nope_lo[th * nope + k] = __float2bfloat16_rn(v - __bfloat162float(h));
+    } else {
+      const int pr = k - nope;
+      const double ang = (double)pos[t] * rope_inv_freq(theta, pr, d_r);
+      double sn, cs;
+      sincos(ang, &sn, &cs);
+      const double r0 = src[nope + 2 * pr], r1 = src[nope + 2 * pr + 1];
+      q_rope[th * d_r + 2 * pr] = (float)(r0 * cs - r1 * sn);
+      q_rope[th * d_r + 2 * pr + 1] = (float)(r0 * sn + r1 * cs);
     }
   }
 }

@@ -22,7 +22,9 @@ struct GemmSimtArgs {
 
 constexpr int kSimtTile = 32;
 
-template <typename TA, typename TB, typename Acc>
+// kAtomic: add the result into C with atomics instead of storing it (split-K
+// partials summed in place; C must start at zero).
+template <typename TA, typename TB, typename Acc, bool kAtomic = false>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmSimtArgs g) {
   __shared__ Acc As[kSimtTile][kSimtTile + 1];
   __shared__ Acc Bs[kSimtTile][kSimtTile + 1];
@@ -53,15 +55,18 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmSimtArgs g) {
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     const int m = m0 + ty + 8 * r, n = n0 + tx;
-    if (m < g.M && n < g.N) C[m * g.sCm + n * g.sCn] = acc[r];
+    if (m < g.M && n < g.N) {
+      if constexpr (kAtomic) atomicAdd(&C[m * g.sCm + n * g.sCn], acc[r]);
+      else C[m * g.sCm + n * g.sCn] = acc[r];
+    }
   }
 }
 
-template <typename TA, typename TB, typename Acc>
+template <typename TA, typename TB, typename Acc, bool kAtomic = false>
 static cudaError_t gemm_simt(const GemmSimtArgs& g, cudaStream_t s) {
   if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return cudaSuccess;
   dim3 grid((g.N + kSimtTile - 1) / kSimtTile, (g.M + kSimtTile - 1) / kSimtTile, g.batch);
-  gemm_simt_kernel<TA, TB, Acc><<<grid, 256, 0, s>>>(g);
+  gemm_simt_kernel<TA, TB, Acc, kAtomic><<<grid, 256, 0, s>>>(g);
   note_launch();
   return cudaGetLastError();
 }

@@ -12,6 +12,7 @@
 #include "decode_tc.cuh"
 #include "elementwise.cuh"
 #include "gemm_simt.cuh"
+#include "wgemm_tc.cuh"
 
 using namespace mla;
 
@@ -52,6 +53,20 @@ int device_sm_count() {
 }
 
 // ---------------------------------------------------------------- append
+// The latent projection is accumulated in fp64 (exact products of bf16
+// values, fp64 sums), so rounding it once gives the bf16 of the real-number
+// dot product.  K is cut into `append_splits` chunks (more parallel work for
+// a skinny GEMM) whose fp64 sums are added into one zeroed fp64 buffer.
+int append_splits(const mla_config* c) {
+  int S = 1;
+  for (int cand = 32; cand > 1; --cand)
+    if (c->hidden % cand == 0 && c->hidden / cand >= 128) {
+      S = cand;
+      break;
+    }
+  return S;
+}
+
 size_t append_ws(const mla_config* c, int n_tok) {
   return align_up(sizeof(double) * (size_t)n_tok * (c->d_c + c->d_r), 256);
 }
@@ -61,12 +76,16 @@ mla_status append_impl(const mla_config* c, const void* x, int n, const void* W_
                        const int32_t* seq_idx, const int32_t* pos, const mla_cache* k, void* ws,
                        cudaStream_t s) {
   const int row = c->d_c + c->d_r;
+  const int S = append_splits(c), Kc = c->hidden / S;
   double* C = static_cast<double*>(ws);
-  MLA_CUDA((gemm_rm<T, T, double>(x, c->hidden, W_DKV, c->d_c, C, row, n, c->d_c, c->hidden, s)));
-  MLA_CUDA((gemm_rm<T, T, double>(x, c->hidden, W_KR, c->d_r, C + c->d_c, row, n, c->d_r, c->hidden, s)));
+  MLA_CUDA(cudaMemsetAsync(C, 0, sizeof(double) * (size_t)n * row, s));
+  GemmSimtArgs g1{x, W_DKV, C, n, c->d_c, Kc, S, c->hidden, 1, Kc, c->d_c, 1, (long long)Kc * c->d_c, row, 1, 0};
+  MLA_CUDA((gemm_simt<T, T, double, true>(g1, s)));
+  GemmSimtArgs g2{x, W_KR, C + c->d_c, n, c->d_r, Kc, S, c->hidden, 1, Kc, c->d_r, 1, (long long)Kc * c->d_r, row, 1, 0};
+  MLA_CUDA((gemm_simt<T, T, double, true>(g2, s)));
   const long long total = (long long)n * (c->d_c + c->d_r / 2);
   append_finish_kernel<T><<<grid_for(total), 256, 0, s>>>(
-      C, n, c->d_c, c->d_r, c->rope_theta, seq_idx, pos, static_cast<T*>(k->pool), k->block_table,
+      C, 1, n, c->d_c, c->d_r, c->rope_theta, seq_idx, pos, static_cast<T*>(k->pool), k->block_table,
       k->batch, k->max_blocks_per_seq, k->num_blocks, c->block_size);
   note_launch();
   return st(cudaGetLastError());
@@ -150,6 +169,121 @@ mla_status out_impl(const mla_config* c, const float* o_lat, int n, const void* 
   MLA_CUDA((gemm_rm<float, T, float>(oh_f, (long long)H * dv, W_O, c->hidden, y_f, c->hidden, n, c->hidden, H * dv, s)));
   MLA_CUDA(round_store<T>(y_f, static_cast<T*>(y), (long long)n * c->hidden, s));
   return MLA_OK;
+}
+
+// ---------------------------------------------------------------- bf16 projections
+// Tensor-core path of the query and output projections (weights bf16; see
+// wgemm_tc.cuh).  Activations enter the MMAs in bf16; with the split-query
+// flag the fp32 query intermediates enter as a bf16 hi + lo pair.
+bool proj_tc_supported(const mla_config* c) {
+  const long long qw = (long long)c->n_heads * (c->qk_nope + c->d_r);
+  return c->hidden % 128 == 0 && (c->q_lora == 0 || c->q_lora % 128 == 0) && qw % 128 == 0 &&
+         c->qk_nope % 64 == 0 && c->d_c % 128 == 0 && c->v_head % 128 == 0;
+}
+
+const bf16* const kSizeOnly = reinterpret_cast<const bf16*>(256);  // placeholder pointer for size queries
+
+struct ProjSpecs {
+  wg::Spec dq, uq, uk, uv, o;
+};
+
+ProjSpecs proj_specs(const mla_config* c, int n, bool split, const void* W_DQ, const void* W_UQ,
+                     const void* W_UK, const void* W_UV, const void* W_O, const bf16* x, const bf16* cq_hi,
+                     const bf16* cq_lo, const bf16* qn_hi, const bf16* qn_lo, const bf16* ol, const bf16* oh) {
+  const int H = c->n_heads, nope = c->qk_nope, qw = H * (c->qk_nope + c->d_r);
+  ProjSpecs p{};
+  p.dq = wg::Spec{static_cast<const bf16*>(W_DQ), c->hidden, c->q_lora, 0, 1, c->q_lora, c->hidden, 0,
+                  x, nullptr, c->hidden, 0, n};
+  const int kq = c->q_lora > 0 ? c->q_lora : c->hidden;
+  p.uq = wg::Spec{static_cast<const bf16*>(W_UQ), kq, qw, 0, 1, qw, kq, 0,
+                  c->q_lora > 0 ? cq_hi : x, c->q_lora > 0 && split ? cq_lo : nullptr, kq, 0, n};
+  p.uk = wg::Spec{static_cast<const bf16*>(W_UK), c->d_c, (long long)H * nope, 1, H, c->d_c, nope, nope,
+                  qn_hi, split ? qn_lo : nullptr, (long long)H * nope, nope, n};
+  p.uv = wg::Spec{static_cast<const bf16*>(W_UV), c->d_c, (long long)H * c->v_head, 0, H, c->v_head, c->d_c,
+                  c->v_head, ol, nullptr, (long long)H * c->d_c, c->d_c, n};
+  p.o = wg::Spec{static_cast<const bf16*>(W_O), (long long)H * c->v_head, c->hidden, 0, 1, c->hidden,
+                 H * c->v_head, 0, oh, nullptr, (long long)H * c->v_head, 0, n};
+  return p;
+}
+
+struct AbsorbTcWs {
+  size_t part, cq_hi, cq_lo, q_f, qn_hi, qn_lo, total;
+};
+AbsorbTcWs absorb_tc_ws(const mla_config* c, int n) {
+  const bool split = (c->flags & MLA_FLAG_SPLIT_QUERY) != 0;
+  const ProjSpecs ps = proj_specs(c, n, split, nullptr, nullptr, nullptr, nullptr, nullptr, kSizeOnly, kSizeOnly,
+                                  kSizeOnly, kSizeOnly, kSizeOnly, kSizeOnly, kSizeOnly);
+  const size_t H = c->n_heads, qw = H * (c->qk_nope + c->d_r);
+  size_t part = wg::run_partial_bytes(ps.uq);
+  part = std::max(part, wg::run_partial_bytes(ps.uk));
+  if (c->q_lora > 0) part = std::max(part, wg::run_partial_bytes(ps.dq));
+  AbsorbTcWs w{};
+  size_t o = 0;
+  w.part = o;  o = align_up(o + part, 256);
+  w.cq_hi = o; o = align_up(o + 2 * (size_t)n * c->q_lora, 256);
+  w.cq_lo = o; o = align_up(o + (split ? 2 * (size_t)n * c->q_lora : 0), 256);
+  w.q_f = o;   o = align_up(o + 4 * (size_t)n * qw, 256);
+  w.qn_hi = o; o = align_up(o + 2 * (size_t)n * H * c->qk_nope, 256);
+  w.qn_lo = o; o = align_up(o + (split ? 2 * (size_t)n * H * c->qk_nope : 0), 256);
+  w.total = o;
+  return w;
+}
+
+mla_status absorb_tc(const mla_config* c, const void* x, int n, const void* W_DQ, const void* W_UQ,
+                     const void* W_UK, const int32_t* pos, float* q_lat, float* q_rope, void* ws, cudaStream_t s) {
+  const bool split = (c->flags & MLA_FLAG_SPLIT_QUERY) != 0;
+  const AbsorbTcWs w = absorb_tc_ws(c, n);
+  char* base = static_cast<char*>(ws);
+  float* part = reinterpret_cast<float*>(base + w.part);
+  bf16* cq_hi = reinterpret_cast<bf16*>(base + w.cq_hi);
+  bf16* cq_lo = split ? reinterpret_cast<bf16*>(base + w.cq_lo) : nullptr;
+  float* q_f = reinterpret_cast<float*>(base + w.q_f);
+  bf16* qn_hi = reinterpret_cast<bf16*>(base + w.qn_hi);
+  bf16* qn_lo = split ? reinterpret_cast<bf16*>(base + w.qn_lo) : nullptr;
+  const ProjSpecs ps = proj_specs(c, n, split, W_DQ, W_UQ, W_UK, nullptr, nullptr, static_cast<const bf16*>(x),
+                                  cq_hi, cq_lo, qn_hi, qn_lo, nullptr, nullptr);
+  if (c->q_lora > 0) MLA_TRY(wg::run(ps.dq, part, nullptr, cq_hi, cq_lo, s));
+  MLA_TRY(wg::run(ps.uq, part, q_f, nullptr, nullptr, s));
+  const int H = c->n_heads, nope = c->qk_nope;
+  const long long tot = (long long)n * H * (nope + c->d_r / 2);
+  query_split_bf16_kernel<<<grid_for(tot), 256, 0, s>>>(q_f, n, H, nope, c->d_r, c->rope_theta, pos, qn_hi, qn_lo,
+                                                        q_rope);
+  note_launch();
+  MLA_CUDA(cudaGetLastError());
+  return wg::run(ps.uk, part, q_lat, nullptr, nullptr, s);
+}
+
+struct OutTcWs {
+  size_t part, ol, oh, total;
+};
+OutTcWs out_tc_ws(const mla_config* c, int n) {
+  const ProjSpecs ps = proj_specs(c, n, false, nullptr, nullptr, nullptr, nullptr, nullptr, kSizeOnly, kSizeOnly,
+                                  kSizeOnly, kSizeOnly, kSizeOnly, kSizeOnly, kSizeOnly);
+  const size_t H = c->n_heads;
+  OutTcWs w{};
+  size_t o = 0;
+  w.part = o; o = align_up(o + std::max(wg::run_partial_bytes(ps.uv), wg::run_partial_bytes(ps.o)), 256);
+  w.ol = o;   o = align_up(o + 2 * (size_t)n * H * c->d_c, 256);
+  w.oh = o;   o = align_up(o + 2 * (size_t)n * H * c->v_head, 256);
+  w.total = o;
+  return w;
+}
+
+mla_status out_tc(const mla_config* c, const float* o_lat, int n, const void* W_UV, const void* W_O, void* y,
+                  void* ws, cudaStream_t s) {
+  const OutTcWs w = out_tc_ws(c, n);
+  char* base = static_cast<char*>(ws);
+  float* part = reinterpret_cast<float*>(base + w.part);
+  bf16* ol = reinterpret_cast<bf16*>(base + w.ol);
+  bf16* oh = reinterpret_cast<bf16*>(base + w.oh);
+  const long long cnt = (long long)n * c->n_heads * c->d_c;
+  wg::split_bf16_kernel<<<grid_for(cnt), 256, 0, s>>>(o_lat, cnt, ol, nullptr);
+  note_launch();
+  MLA_CUDA(cudaGetLastError());
+  const ProjSpecs ps = proj_specs(c, n, false, nullptr, nullptr, nullptr, W_UV, W_O, nullptr, nullptr, nullptr,
+                                  nullptr, nullptr, ol, oh);
+  MLA_TRY(wg::run(ps.uv, part, nullptr, oh, nullptr, s));
+  return wg::run(ps.o, part, nullptr, static_cast<bf16*>(y), nullptr, s);
 }
 
 // ---------------------------------------------------------------- decode
@@ -273,8 +407,8 @@ mla_status mla_cache_append_noalloc(const mla_config* cfg, const void* x, int32_
   if (need > (size_t)MLA_APPEND_NOALLOC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
   void* scratch = nullptr;
   MLA_TRY(append_scratch_address(&scratch));
-  // Every value of the scratch that the append reads is written first by the
-  // same call, so nothing left over from an earlier call needs clearing.
+  // The append clears the part of the scratch it accumulates into at the start
+  // of every call, so nothing left over from an earlier call leaks in.
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cfg->dtype == MLA_BF16)
     return append_impl<bf16>(cfg, x, n_tok, W_DKV, W_KR, seq_idx, pos, cache, scratch, s);
@@ -283,6 +417,7 @@ mla_status mla_cache_append_noalloc(const mla_config* cfg, const void* x, int32_
 
 size_t mla_absorb_q_workspace_size(const mla_config* cfg, int32_t n_tok) {
   if (check_cfg(cfg) != MLA_OK || n_tok < 0) return 0;
+  if (cfg->dtype == MLA_BF16) return proj_tc_supported(cfg) ? absorb_tc_ws(cfg, n_tok).total : 0;
   return absorb_ws(cfg, n_tok).total;
 }
 
@@ -294,10 +429,13 @@ mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok, con
   if (n_tok == 0) return MLA_OK;
   if (!x || !W_UQ || !W_UK || !pos || !q_lat || !q_rope || !workspace) return MLA_ERR_INVALID_ARG;
   if ((cfg->q_lora > 0) != (W_DQ != nullptr)) return MLA_ERR_INVALID_ARG;
-  if (ws_bytes < absorb_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cfg->dtype == MLA_BF16)
-    return absorb_impl<bf16>(cfg, x, n_tok, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, workspace, s);
+  if (cfg->dtype == MLA_BF16) {
+    if (!proj_tc_supported(cfg)) return MLA_ERR_UNSUPPORTED;
+    if (ws_bytes < absorb_tc_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
+    return absorb_tc(cfg, x, n_tok, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, workspace, s);
+  }
+  if (ws_bytes < absorb_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
   return absorb_impl<float>(cfg, x, n_tok, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, workspace, s);
 }
 
@@ -350,6 +488,7 @@ mla_status mla_combine(const mla_config* cfg, const void* workspace, size_t ws_b
 
 size_t mla_out_proj_workspace_size(const mla_config* cfg, int32_t n_tok) {
   if (check_cfg(cfg) != MLA_OK || n_tok < 0) return 0;
+  if (cfg->dtype == MLA_BF16) return proj_tc_supported(cfg) ? out_tc_ws(cfg, n_tok).total : 0;
   return out_ws(cfg, n_tok).total;
 }
 
@@ -359,9 +498,13 @@ mla_status mla_out_proj(const mla_config* cfg, const float* o_lat, int32_t n_tok
   if (n_tok < 0) return MLA_ERR_INVALID_ARG;
   if (n_tok == 0) return MLA_OK;
   if (!o_lat || !W_UV || !W_O || !y || !workspace) return MLA_ERR_INVALID_ARG;
-  if (ws_bytes < out_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cfg->dtype == MLA_BF16) return out_impl<bf16>(cfg, o_lat, n_tok, W_UV, W_O, y, workspace, s);
+  if (cfg->dtype == MLA_BF16) {
+    if (!proj_tc_supported(cfg)) return MLA_ERR_UNSUPPORTED;
+    if (ws_bytes < out_tc_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
+    return out_tc(cfg, o_lat, n_tok, W_UV, W_O, y, workspace, s);
+  }
+  if (ws_bytes < out_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
   return out_impl<float>(cfg, o_lat, n_tok, W_UV, W_O, y, workspace, s);
 }
 

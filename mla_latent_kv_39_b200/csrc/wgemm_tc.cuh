@@ -1,0 +1,408 @@
+// Weight-streaming GEMM on the sm_100 tensor cores (tcgen05 + TMEM + TMA).
+//
+// C[g][t][f] = sum_k X[t][g][k] W_g[k][f] for the projections of the decode
+// step, where the weights (hundreds of MB) dominate the bytes and the tokens
+// are few (a decode batch).  So the MMA runs "swap AB": 128 output features
+// of W are the M side (A operand), the tokens the N side (B operand, N <= 256),
+// and the weights stream through shared memory once.  The K dimension is cut
+// into S splits so that every SM streams its share; each (group, feature tile,
+// split) writes an fp32 partial, and a separate pass sums the splits in a fixed
+// order (deterministic results) and applies the step's epilogue.
+//
+// A (weights, bf16) comes in two layouts:
+//   MN-major: W stored [K, F] (features contiguous)  -> two 64-feature TMA boxes
+//   K-major : W stored [F, K] (K contiguous; W_UK)    -> one 128-row TMA box
+// B (activations, bf16, K contiguous) is a 3-D view [tokens, groups, K]; with
+// `split` a second view holds the bf16 remainder (lo) of fp32 activations and
+// both are accumulated against the same weights.
+//
+// Roles (192 threads): warp 0 TMA, warp 1 TMEM allocation + MMA issue, warps
+// 2-5 read the accumulator (two TMEM buffers of 256 columns, so the drain of
+// one work item overlaps the MMAs of the next).
+#pragma once
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace mla {
+namespace wg {
+
+using namespace sm100;
+
+constexpr int kStages = 4;
+constexpr int kABytes = 128 * 128;            // 128 features x 64 k, bf16
+constexpr int kStageBytes = 48 * 1024;        // A + up to 256 x 64 (or 2 x 128 x 64) of B
+constexpr int kThreads = 192;
+
+struct Smem {
+  uint8_t stage[kStages][kStageBytes];  // first member: 1024-byte aligned
+  uint64_t full[kStages], empty[kStages];
+  uint64_t acc_full[2], acc_empty[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+
+struct Params {
+  int G, MT, KB, S;     // groups, 128-feature tiles per group, 64-k blocks per group, K splits
+  int n_tok, N;         // tokens, MMA N (tokens rounded up to 16)
+  int a_kmajor;         // A layout (see above)
+  int a_g_stride;       // MN-major: feature offset per group; K-major: k offset per group
+  int split;            // B has a lo part
+  int F;                // features per group
+  float* part;          // [S][n_tok][G][F]
+};
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void item_coords(const Params& p, int item, int& g, int& mt, int& kb0, int& kb1, int& s) {
+  const int per_g = p.MT * p.S;
+  g = item / per_g;
+  const int rem = item % per_g;
+  mt = rem / p.S;
+  s = rem % p.S;
+  kb0 = (int)((long long)s * p.KB / p.S);
+  kb1 = (int)((long long)(s + 1) * p.KB / p.S);
+}
+
+__device__ __forceinline__ void set_abort(Smem& sm) { *(volatile int*)&sm.abort_flag = 1; }
+__device__ __forceinline__ bool aborted(Smem& sm) { return *(volatile int*)&sm.abort_flag != 0; }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    wgemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap_hi,
+                 const __grid_constant__ CUtensorMap bmap_lo, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int items = p.G * p.MT * p.S;
+  const uint32_t b_bytes = (uint32_t)p.N * 128u;
+  const uint32_t stage_tx = (uint32_t)kABytes + b_bytes * (p.split ? 2u : 1u);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.acc_full[b], 1);
+      mbar_init(&sm.acc_empty[b], 128);
+    }
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&amap);
+    prefetch_tensormap(&bmap_hi);
+    if (p.split) prefetch_tensormap(&bmap_lo);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int k = 0;
+      for (int item = blockIdx.x; item < items && !aborted(sm); item += gridDim.x) {
+        int g, mt, kb0, kb1, s;
+        item_coords(p, item, g, mt, kb0, kb1, s);
+        for (int kb = kb0; kb < kb1; ++kb, ++k) {
+          const int st = k % kStages;
+          if (k >= kStages && !mbar_wait(&sm.empty[st], ((k / kStages) - 1) & 1, 70)) {
+            set_abort(sm);
+            goto producer_drain;
+          }
+          uint8_t* a = sm.stage[st];
+          uint8_t* b = a + kABytes;
+          mbar_arrive_expect_tx(&sm.full[st], stage_tx);
+          if (p.a_kmajor) {
+            tma_load_2d(a, &amap, g * p.a_g_stride + kb * 64, mt * 128, &sm.full[st]);
+          } else {
+            tma_load_2d(a, &amap, g * p.a_g_stride + mt * 128, kb * 64, &sm.full[st]);
+            tma_load_2d(a + kABytes / 2, &amap, g * p.a_g_stride + mt * 128 + 64, kb * 64, &sm.full[st]);
+          }
+          tma_load_3d(b, &bmap_hi, kb * 64, g, 0, &sm.full[st]);
+          if (p.split) tma_load_3d(b + b_bytes, &bmap_lo, kb * 64, g, 0, &sm.full[st]);
+        }
+      }
+    producer_drain:
+      for (int kk = k - kStages < 0 ? 0 : k - kStages; kk < k; ++kk)
+        mbar_wait(&sm.full[kk % kStages], (kk / kStages) & 1, 71);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      const uint32_t idesc = idesc_bf16_f32(128, p.N, p.a_kmajor ? 0 : 1, 0);
+      // A: MN-major -> 64-feature chunks 8 KiB apart (LBO), 8 k-rows 1 KiB apart
+      // (SBO), K step j at +2 KiB * j; K-major -> rows 128 B apart, 8-row groups
+      // 1 KiB apart (SBO), K step j at +32 B * j.  B: K-major like the latter.
+      const uint64_t a0 = p.a_kmajor ? smem_desc(smem_u32(sm.stage[0]), 16, 1024, kSwizzle128B)
+                                     : smem_desc(smem_u32(sm.stage[0]), kABytes / 2, 1024, kSwizzle128B);
+      const uint64_t b0 = smem_desc(smem_u32(sm.stage[0]) + kABytes, 16, 1024, kSwizzle128B);
+      int k = 0, j = 0;
+      for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+        int g, mt, kb0, kb1, s;
+        item_coords(p, item, g, mt, kb0, kb1, s);
+        const int buf = j & 1;
+        if (j >= 2 && !mbar_wait(&sm.acc_empty[buf], ((j >> 1) - 1) & 1, 72)) goto mma_fail;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * 256;
+        for (int kb = kb0; kb < kb1; ++kb, ++k) {
+          const int st = k % kStages;
+          if (!mbar_wait(&sm.full[st], (k / kStages) & 1, 73)) goto mma_fail;
+          tc_fence_after();
+          const uint32_t so = (uint32_t)(st * kStageBytes) >> 4;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint64_t ad = a0 + so + ((p.a_kmajor ? q * 32u : q * 2048u) >> 4);
+            const uint64_t bd = b0 + so + ((q * 32u) >> 4);
+            mma_ss(d, ad, bd, idesc, (kb > kb0 || q > 0) ? 1u : 0u);
+            if (p.split) mma_ss(d, ad, bd + (b_bytes >> 4), idesc, 1u);
+          }
+          mma_commit(&sm.empty[st]);
+        }
+        mma_commit(&sm.acc_full[buf]);
+      }
+      goto mma_end;
+    mma_fail:
+      set_abort(sm);
+    mma_end:;
+    }
+  } else {
+    // ------------------------------------------------ accumulator drain
+    const int qw = warp & 3;
+    const int f_local = qw * 32 + lane;  // feature within the 128-wide tile == TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);
+    int j = 0;
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
+      int g, mt, kb0, kb1, s;
+      item_coords(p, item, g, mt, kb0, kb1, s);
+      const int buf = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.acc_full[buf], (j >> 1) & 1, 74))) {
+        set_abort(sm);
+        break;
+      }
+      tc_fence_after();
+      const long long tstride = (long long)p.G * p.F;
+      float* out = p.part + (long long)s * p.n_tok * tstride + (long long)g * p.F + mt * 128 + f_local;
+      for (int c = 0; c < p.N; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tl + buf * 256 + c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 32; ++t)
+          if (c + t < p.n_tok) out[(long long)(c + t) * tstride] = __uint_as_float(v[t]);
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.acc_empty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// out[i] = sum_s part[s][i] over `count` elements, written as fp32 and/or bf16
+// (hi) and/or the bf16 remainder (lo = value - hi).
+__global__ void reduce_splits_kernel(const float* __restrict__ part, int S, long long count, float* out_f32,
+                                     bf16* out_hi, bf16* out_lo) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
+       i += (long long)gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < S; ++s) acc += part[(long long)s * count + i];
+    if (out_f32) out_f32[i] = acc;
+    if (out_hi) {
+      const bf16 h = __float2bfloat16_rn(acc);
+      out_hi[i] = h;
+      if (out_lo) out_lo[i] = __float2bfloat16_rn(acc - __bfloat162float(h));
+    }
+  }
+}
+
+// fp32 -> bf16 (hi) and optional remainder (lo).
+__global__ void split_bf16_kernel(const float* __restrict__ in, long long count, bf16* out_hi, bf16* out_lo) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float v = in[i];
+    const bf16 h = __float2bfloat16_rn(v);
+    out_hi[i] = h;
+    if (out_lo) out_lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+}  // namespace wg
+}  // namespace mla
+
+// ================================================================ host side
+namespace mla {
+namespace wg {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_tiled() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load(std::memory_order_acquire);
+  if (f == nullptr) {
+    void* q = nullptr;
+    cudaDriverEntryPointQueryResult r;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess && q != nullptr) {
+      f = reinterpret_cast<EncodeTiledFn>(q);
+      fn.store(f, std::memory_order_release);
+    }
+  }
+  return f;
+}
+
+// One projection of the step: weights W (bf16, as stored) against bf16
+// activations B[t][g][k] (element t * b_t_stride + g * b_g_stride + k).
+struct Spec {
+  const bf16* W;
+  long long w_rows, w_cols;  // W as stored, row-major
+  int a_kmajor;              // 0: W is [K, features]; 1: W is [features, K]
+  int G, F, Kg;              // groups, features per group (x128), K per group (x64)
+  int a_g_stride;            // MN-major: feature column offset of group g; K-major: k column offset
+  const bf16* B_hi;
+  const bf16* B_lo;          // optional bf16 remainder of fp32 activations
+  long long b_t_stride, b_g_stride;
+  int n_tok;                 // tokens of this call (<= 256)
+};
+
+inline bool spec_ok(const Spec& s) {
+  return s.F % 128 == 0 && s.Kg % 64 == 0 && s.n_tok > 0 && s.G > 0;
+}
+
+// Tokens per launch: the MMA N is at most 256, and a stage holds 256 token
+// rows of one activation view (128 rows each of hi and lo).
+inline int max_chunk(const Spec& s) { return s.B_lo ? 128 : 256; }
+
+// K splits: enough work items to fill the SMs twice, while the partial sums
+// stay small next to the weights they come from.
+inline int choose_splits(const Spec& s, int sms) {
+  const int MT = s.F / 128, KB = s.Kg / 64;
+  const long long base = (long long)s.G * MT;
+  int S = (int)std::max<long long>(1, std::min<long long>(KB, (2LL * sms + base - 1) / base));
+  const double wbytes = 2.0 * s.G * (double)s.F * s.Kg;
+  const double out_bytes = 4.0 * s.G * (double)s.F * s.n_tok;
+  while (S > 1 && (S * out_bytes > 0.25 * wbytes || KB / S < 2)) --S;
+  return S;
+}
+
+inline size_t partial_floats(const Spec& s, int S) {
+  return (size_t)S * std::min(s.n_tok, max_chunk(s)) * s.G * s.F;
+}
+
+inline int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 148;
+  return n > 0 ? n : 148;
+}
+
+inline mla_status make_maps(const Spec& s, int N, CUtensorMap* a, CUtensorMap* bh, CUtensorMap* bl) {
+  EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return MLA_ERR_CUDA;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)s.w_cols, (cuuint64_t)s.w_rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)s.w_cols * 2};
+    const cuuint32_t box[2] = {64, s.a_kmajor ? 128u : 64u};
+    const cuuint32_t es[2] = {1, 1};
+    if (enc(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)s.W, dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  }
+  const bf16* srcs[2] = {s.B_hi, s.B_lo};
+  CUtensorMap* maps[2] = {bh, bl};
+  for (int i = 0; i < 2; ++i) {
+    const bf16* src = srcs[i] ? srcs[i] : s.B_hi;
+    const cuuint64_t dims[3] = {(cuuint64_t)s.Kg, (cuuint64_t)s.G, (cuuint64_t)s.n_tok};
+    const cuuint64_t strides[2] = {(cuuint64_t)(s.G > 1 ? s.b_g_stride : s.Kg) * 2, (cuuint64_t)s.b_t_stride * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)N};
+    const cuuint32_t es[3] = {1, 1, 1};
+    if (enc(maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)src, dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
+inline mla_status set_attr() {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return MLA_OK;
+  if (cudaFuncSetAttribute(wgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return MLA_OK;
+}
+
+// Projection into fp32 partials [S][n_tok][G][F], then their sum into the
+// requested outputs (fp32 and/or bf16 hi and/or bf16 lo), all [n_tok][G][F].
+inline mla_status run(const Spec& s0, float* part, float* out_f32, bf16* out_hi, bf16* out_lo, cudaStream_t st) {
+  if (!spec_ok(s0)) return MLA_ERR_UNSUPPORTED;
+  const int chunk = max_chunk(s0);
+  if (s0.n_tok > chunk) {
+    for (int t0 = 0; t0 < s0.n_tok; t0 += chunk) {
+      Spec c = s0;
+      c.n_tok = std::min(chunk, s0.n_tok - t0);
+      c.B_hi = s0.B_hi + (long long)t0 * s0.b_t_stride;
+      c.B_lo = s0.B_lo ? s0.B_lo + (long long)t0 * s0.b_t_stride : nullptr;
+      const long long o = (long long)t0 * s0.G * s0.F;
+      const mla_status ms = run(c, part, out_f32 ? out_f32 + o : nullptr, out_hi ? out_hi + o : nullptr,
+                                out_lo ? out_lo + o : nullptr, st);
+      if (ms != MLA_OK) return ms;
+    }
+    return MLA_OK;
+  }
+  const Spec& s = s0;
+  const int sms = device_sms();
+  const int S = choose_splits(s, sms);
+  const int N = (s.n_tok + 15) / 16 * 16;
+  if (((uintptr_t)s.W & 15u) || ((uintptr_t)s.B_hi & 15u) || (s.B_lo && ((uintptr_t)s.B_lo & 15u)))
+    return MLA_ERR_INVALID_ARG;
+  CUtensorMap a, bh, bl;
+  mla_status ms = make_maps(s, N, &a, &bh, &bl);
+  if (ms != MLA_OK) return ms;
+  if ((ms = set_attr()) != MLA_OK) return ms;
+  Params p{s.G, s.F / 128, s.Kg / 64, S, s.n_tok, N, s.a_kmajor, s.a_g_stride, s.B_lo ? 1 : 0, s.F, part};
+  const int items = s.G * (s.F / 128) * S;
+  wgemm_kernel<<<std::min(items, sms), kThreads, kSmemBytes, st>>>(a, bh, bl, p);
+  note_launch();
+  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  const long long count = (long long)s.n_tok * s.G * s.F;
+  const int blocks = (int)std::min<long long>((count + 255) / 256, 4 * sms);
+  reduce_splits_kernel<<<blocks, 256, 0, st>>>(part, S, count, out_f32, out_hi, out_lo);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+inline size_t run_partial_bytes(const Spec& s0) {
+  if (!spec_ok(s0)) return 0;
+  Spec s = s0;
+  s.n_tok = std::min(s0.n_tok, max_chunk(s0));
+  return partial_floats(s, choose_splits(s, device_sms())) * sizeof(float);
+}
+
+}  // namespace wg
+}  // namespace mla

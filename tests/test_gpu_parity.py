@@ -42,10 +42,13 @@ SMALL_CASES = [
     ("v3_b64_ragged1k_8k", [700, 1, 130, 191, 257, 64], None),
     ("v3_b4_long", [5000, 20000], None),
     ("v3_b128_nq2_ragged512_16k", [0, 1, 62, 63, 64, 300], 2),
+    # 260 new tokens: the projections run in two token chunks
+    ("v3_b128_nq2_ragged512_16k", [3] * 130, 2),
 ]
 
 
-@pytest.mark.parametrize("name,lengths,n_q", SMALL_CASES, ids=[c[0] for c in SMALL_CASES])
+@pytest.mark.parametrize("name,lengths,n_q", SMALL_CASES,
+                         ids=[f"{c[0]}-{i}" for i, c in enumerate(SMALL_CASES)])
 def test_small_cases_every_element(name, lengths, n_q):
     wl = reduced(WORKLOADS[name], lengths=lengths, n_q=n_q)
     data, dev, layer = run_gpu(wl)
