@@ -6,12 +6,11 @@
 //  * two score tiles in TMEM; P (bf16) is written over the score tile it came
 //    from, so the MMA warp computes the scores of page k+1 (and k+2) while the
 //    softmax works on page k, and a P store never waits for the previous P V;
-//  * the partial scores of page k+1 are sent to the peer before page k is
-//    processed, so the exchange latency hides behind a page of work: each
-//    softmax warp stages its 32 x 32 block in local shared memory and one
-//    lane ships it with a 4 KiB bulk copy into the peer's shared memory,
-//    counted in bytes on the peer's mbarrier; each CTA tells the peer when it
-//    has read a buffer (xempty) before the peer refills it;
+//  * the partial scores of page k+1 go to the peer as soon as they exist -
+//    before page k is processed when the MMA warp is ahead - through st.async
+//    stores into the peer's shared memory, counted in bytes on the peer's
+//    mbarrier (no fence); each CTA tells the peer when it has read a buffer
+//    (xempty, a relaxed remote arrive) before the peer refills it;
 //  * eight softmax warps: the two warps of a TMEM lane quarter split the 64
 //    tokens of a page (32 each) and meet once per page to agree on the row max;
 //  * the producer prefetches pages into L2 several pages ahead of the shared
@@ -35,7 +34,7 @@ using namespace sm100;
 
 constexpr int kH = 128, kDc = 512, kDr = 64, kBS = 64;
 constexpr int kSlabBytes = 64 * 128;                 // 64 rows x 64 bf16 (128 B), swizzled
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kPrefetch = 8;                         // pages prefetched into L2 ahead of the stages
 constexpr int kStageBytes = 5 * kSlabBytes;          // 40 KiB (CTA 0 uses 4 slabs)
 constexpr int kQropeBytes = 128 * 128;               // 128 rows x 64 bf16, swizzled
@@ -52,7 +51,6 @@ struct Smem {
   // Exchanged partial scores: one 4 KiB block per softmax warp (32 rows x 32
   // tokens); the 16-byte chunk c of a row sits at chunk position c ^ (row & 7).
   float xrecv[2][kSoftmaxWarps][32][32];  // from the peer, per score buffer
-  float xsend[kSoftmaxWarps][32][32];     // staging of this CTA's block for the peer
   float rowx[2][4][2][32];           // per page parity, lane quarter, column half: partial max
   float rowl[4][2][32];              // partial row sums at a segment's end
   uint64_t full[kStages], empty[kStages];
@@ -79,20 +77,12 @@ struct Params {
 __device__ __forceinline__ void set_abort(Smem& sm) { *(volatile int*)&sm.abort_flag = 1; }
 __device__ __forceinline__ bool aborted(Smem& sm) { return *(volatile int*)&sm.abort_flag != 0; }
 
-// Bulk copy of `bytes` from this CTA's shared memory into the peer's,
-// counted in bytes on the peer's mbarrier.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_local, uint32_t bytes,
-                                                  uint32_t mbar_cluster) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(dst_cluster), "r"(src_local), "r"(bytes), "r"(mbar_cluster)
-      : "memory");
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Wait until every bulk copy this thread committed has finished reading its source.
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+// 16-byte store into the peer CTA's shared memory, counted in bytes on the
+// peer's mbarrier (no fence: the barrier's transaction count orders it).
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t mbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+               ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(mbar)
+               : "memory");
 }
 
 // Arrive on a barrier of the peer CTA without ordering earlier memory
@@ -295,33 +285,30 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
   const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);  // this warp's lane quarter
   const uint32_t peer = crank ^ 1u;
   const int wi = warp - 2;                                 // softmax warp index 0..7
-  const uint32_t xrecv_peer = mapa(smem_u32(&sm.xrecv[0][wi][0][0]), peer);
-  const uint32_t xsend_local = smem_u32(&sm.xsend[wi][0][0]);
+  const uint32_t xrow_peer = mapa(smem_u32(&sm.xrecv[0][wi][lane][0]), peer);
   const uint32_t xfull_peer[2] = {mapa(smem_u32(&sm.xfull[0]), peer), mapa(smem_u32(&sm.xfull[1]), peer)};
   const uint32_t xempty_peer[2] = {mapa(smem_u32(&sm.xempty[0]), peer), mapa(smem_u32(&sm.xempty[1]), peer)};
   const int xsw = lane & 7;
   float* part_o = ws_at<float>(p.ws, p.L.off_o);
   float* part_lse = ws_at<float>(p.ws, p.L.off_lse);
 
-  // This thread's 32 partial scores of page kk: TMEM -> registers -> this
-  // warp's staging block -> (bulk copy) the peer's buffer kk % 2, once the
-  // peer has read what that buffer held (page kk - 2).
+  // This thread's 32 partial scores of page kk: TMEM -> registers -> the
+  // peer's buffer kk % 2, once the peer has read what it held (page kk - 2).
   auto fetch_and_send = [&](int kk, float (&s)[32]) -> bool {
     const int buf = kk & 1;
     if (!MLA_WARP_WAIT(mbar_wait(&sm.s_full[buf], (kk >> 1) & 1, 60))) return false;
     tc_fence_after();
     load_scores32(tl + kTmemSP + buf * 64 + ch * 32, s);
-    if (lane == 0) bulk_wait_read();  // the previous copy has read the staging block
-    __syncwarp();
-    float4* row = reinterpret_cast<float4*>(&sm.xsend[wi][lane][0]);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) row[c ^ xsw] = make_float4(s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
-    fence_proxy_async_smem();
-    __syncwarp();
     if (kk >= 2 && !MLA_WARP_WAIT(mbar_wait(&sm.xempty[buf], ((kk >> 1) - 1) & 1, 64))) return false;
-    if (lane == 0)
-      bulk_copy_to_peer(xrecv_peer + buf * kXStageBytes, xsend_local, 32 * 32 * 4, xfull_peer[buf]);
+    const uint32_t dst = xrow_peer + buf * kXStageBytes;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      st_async_v4(dst + ((c ^ xsw) * 16), s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3], xfull_peer[buf]);
     return true;
+  };
+  // Whether page kk's scores are already in TMEM (no waiting).
+  auto scores_ready = [&](int kk) -> bool {
+    return __all_sync(0xffffffffu, mbar_test(&sm.s_full[kk & 1], (kk >> 1) & 1));
   };
 
   int k = 0;
@@ -341,6 +328,7 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
     if (!fetch_and_send(k, sa)) goto fail;
     for (int i = 0; i < T; ++i) {
       const int kk = k + i, buf = kk & 1, blk = sg.y + i;
+      bool sent_next = false;
       // the peer's half of page kk (32 KiB counted on this barrier)
       if (tid == 0) mbar_arrive_expect_tx(&sm.xfull[buf], kXStageBytes);
       if (!MLA_WARP_WAIT(mbar_wait(&sm.xfull[buf], (kk >> 1) & 1, 61))) goto fail;
@@ -356,7 +344,12 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
         }
       }
       mbar_arrive_cluster_relaxed(xempty_peer[buf]);  // buffer read: the peer may refill it
-      if (i + 1 < T && !fetch_and_send(kk + 1, sb)) goto fail;
+      // Send the next page's scores now if the MMA warp already has them;
+      // otherwise process this page first and send them afterwards.
+      if (i + 1 < T && scores_ready(kk + 1)) {
+        if (!fetch_and_send(kk + 1, sb)) goto fail;
+        sent_next = true;
+      }
 
       // scale, mask past the sequence end, and the row max over both halves
       const int valid = min(kBS, len_v - blk * kBS) - ch * 32;
@@ -426,6 +419,7 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_ready[buf]);
+      if (i + 1 < T && !sent_next && !fetch_and_send(kk + 1, sb)) goto fail;
 #pragma unroll
       for (int t = 0; t < 32; ++t) sa[t] = sb[t];
     }
@@ -456,10 +450,8 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
     }
     k += T;
   }
-  if (lane == 0) bulk_wait_read();
   return;
 fail:
-  if (lane == 0) bulk_wait_read();
   set_abort(sm);
 }
 
