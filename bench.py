@@ -101,14 +101,20 @@ def recorded_traffic(workload: str):
 
 class ClockSampler:
     """SM clock and throttle reasons of this process's GPU, sampled through NVML
-    (the library nvidia-smi reads) every 20 ms while the timed region runs."""
+    (the library nvidia-smi reads) every 5 ms while the timed region runs."""
 
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index: int, period_s: float = 0.02):
+    def __init__(self, index: int, period_s: float = 0.005):
         self.index, self.period, self.rows, self.err = index, period_s, [], None
+        self.max_mhz = None
         self._stop = threading.Event()
+        try:  # NVML start-up takes longer than a short timed region: do it first
+            self.nv, self.h = self._handle()
+            self.max_mhz = self.nv.nvmlDeviceGetMaxClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report unsampled
+            self.nv, self.err = None, repr(e)
 
     def _handle(self):
         import pynvml
@@ -118,15 +124,17 @@ class ClockSampler:
         return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid)
 
     def _run(self):
+        if self.nv is None:
+            return
+        nv, h = self.nv, self.h
         try:
-            nv, h = self._handle()
-            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-            while not self._stop.is_set():
+            while True:  # at least one sample, even for a very short region
                 sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
                 reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
                 self.rows.append((sm, reasons))
-                self._stop.wait(self.period)
-        except Exception as e:  # no NVML: report unsampled
+                if self._stop.wait(self.period):
+                    break
+        except Exception as e:
             self.err = repr(e)
 
     def __enter__(self):
@@ -361,7 +369,7 @@ def run_ours(args):
 def parse(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))

@@ -37,6 +37,12 @@
  *    a sequence shorter than its query count) skip the offending work,
  *    record the first such error in the device error word, and surface
  *    through mla_get_device_error.  No C++ exception crosses this ABI.
+ *  - Alignment: on the bf16 path, every tensor argument of mla_absorb_q,
+ *    mla_decode, mla_combine and mla_out_proj, and the workspaces, must start
+ *    on a 16-byte boundary (cudaMalloc and PyTorch allocations do); the
+ *    kernels read and write them with TMA and 16-byte vector accesses.  A
+ *    pointer that does not returns MLA_ERR_INVALID_ARG.  mla_cache_append
+ *    takes any alignment (unaligned operands take a slower kernel).
  *  - Storage dtype: MLA_BF16 (bf16 storage, fp32 accumulation) or MLA_F32
  *    (fp32 storage and arithmetic on CUDA cores, for small shapes).
  */

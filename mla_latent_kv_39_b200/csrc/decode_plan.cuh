@@ -221,6 +221,24 @@ __global__ void __launch_bounds__(128) combine_kernel(const void* ws, long long 
   float Z = 0.f;
   for (int s = 0; s < n; ++s) Z += exp2f(lse[(long long)(first + s) * H + h] - M);
   const float invZ = 1.f / Z;
+  const bool vec = (d_c % 4 == 0) && ((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(part)) & 15u) == 0;
+  if (vec) {  // 16-byte loads of the partials, split weights evaluated once per split
+    for (int d = 4 * threadIdx.x; d < d_c; d += 4 * blockDim.x) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int s = 0; s < n; ++s) {
+        const long long r = (long long)(first + s) * H + h;
+        const float wgt = exp2f(lse[r] - M);
+        const float4 p4 = __ldcs(reinterpret_cast<const float4*>(part + r * d_c + d));
+        acc.x += wgt * p4.x;
+        acc.y += wgt * p4.y;
+        acc.z += wgt * p4.z;
+        acc.w += wgt * p4.w;
+      }
+      *reinterpret_cast<float4*>(out + d) = make_float4(acc.x * invZ, acc.y * invZ, acc.z * invZ, acc.w * invZ);
+    }
+    return;
+  }
   for (int d = threadIdx.x; d < d_c; d += blockDim.x) {
     float acc = 0.f;
     for (int s = 0; s < n; ++s) {

@@ -115,33 +115,42 @@ __global__ void query_split_kernel(const float* __restrict__ q, int n_tok, int H
 }
 
 // Split q [n, H, nope + d_r] (fp32): q_nope to bf16 (and its bf16 remainder
-// when lo != nullptr), the rotated q_rope kept in fp32 (angle and rotation in fp64).
+// when lo != nullptr), the rotated q_rope kept in fp32 (angle and rotation in
+// fp64).  One block per (token, group of kHeadGroup heads): the token's d_r/2
+// rotation angles are evaluated once into shared memory and shared by every
+// head.  Needs even nope and d_r (pairs are read and written together).
+constexpr int kHeadGroup = 32;
 __global__ void query_split_bf16_kernel(const float* __restrict__ q, int n_tok, int H, int nope, int d_r,
                                         double theta, const int32_t* __restrict__ pos, bf16* __restrict__ q_nope,
                                         bf16* __restrict__ q_nope_lo, float* __restrict__ q_rope) {
-  const int w = nope + d_r;
-  const int per_head = nope + d_r / 2;
-  const long long total = (long long)n_tok * H * per_head;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long th = i / per_head;
-    const int k = (int)(i % per_head);
-    const int t = (int)(th / H);
-    const float* src = q + th * w;
-    if (k < nope) {
-      const float v = src[k];
-      const bf16 h = __float2bfloat16_rn(v);
-      q_nope[th * nope + k] = h;
-      if (q_nope_lo) q_nope_lo[th * nope + k] = __float2bfloat16_rn(v - __bfloat162float(h));
-    } else {
-      const int pr = k - nope;
-      const double ang = (double)pos[t] * rope_inv_freq(theta, pr, d_r);
-      double sn, cs;
-      sincos(ang, &sn, &cs);
-      const double r0 = src[nope + 2 * pr], r1 = src[nope + 2 * pr + 1];
-      q_rope[th * d_r + 2 * pr] = (float)(r0 * cs - r1 * sn);
-      q_rope[th * d_r + 2 * pr + 1] = (float)(r0 * sn + r1 * cs);
-    }
+  extern __shared__ double rot[];  // [d_r/2][cos, sin]
+  const int t = blockIdx.x, half = d_r / 2, w = nope + d_r;
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    double sn, cs;
+    sincos((double)pos[t] * rope_inv_freq(theta, i, d_r), &sn, &cs);
+    rot[2 * i] = cs;
+    rot[2 * i + 1] = sn;
+  }
+  __syncthreads();
+  const int h0 = blockIdx.y * kHeadGroup, nh = min(kHeadGroup, H - h0);
+  const int np = nope / 2;
+  for (int e = threadIdx.x; e < nh * np; e += blockDim.x) {
+    const long long th = (long long)t * H + h0 + e / np;
+    const int k = 2 * (e % np);
+    const float2 v = *reinterpret_cast<const float2*>(q + th * w + k);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(v.x, v.y);
+    *reinterpret_cast<__nv_bfloat162*>(q_nope + th * nope + k) = hi;
+    if (q_nope_lo)
+      *reinterpret_cast<__nv_bfloat162*>(q_nope_lo + th * nope + k) =
+          __floats2bfloat162_rn(v.x - __bfloat162float(hi.x), v.y - __bfloat162float(hi.y));
+  }
+  for (int e = threadIdx.x; e < nh * half; e += blockDim.x) {
+    const long long th = (long long)t * H + h0 + e / half;
+    const int pr = e % half;
+    const float2 r = *reinterpret_cast<const float2*>(q + th * w + nope + 2 * pr);
+    const double cs = rot[2 * pr], sn = rot[2 * pr + 1];
+    *reinterpret_cast<float2*>(q_rope + th * d_r + 2 * pr) =
+        make_float2((float)((double)r.x * cs - (double)r.y * sn), (float)((double)r.x * sn + (double)r.y * cs));
   }
 }
 

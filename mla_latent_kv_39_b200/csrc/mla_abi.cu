@@ -6,6 +6,7 @@
 #include <cmath>
 #include <mutex>
 
+#include "append_f64.cuh"
 #include "common.cuh"
 #include "decode_plan.cuh"
 #include "decode_simt.cuh"
@@ -34,6 +35,12 @@ mla_status check_cache(const mla_cache* k) {
       k->max_blocks_per_seq <= 0)
     return MLA_ERR_INVALID_ARG;
   return MLA_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+template <typename... P>
+inline bool all_aligned16(const P*... p) {
+  return (aligned16(p) && ...);
 }
 
 inline mla_status st(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
@@ -76,13 +83,23 @@ mla_status append_impl(const mla_config* c, const void* x, int n, const void* W_
                        const int32_t* seq_idx, const int32_t* pos, const mla_cache* k, void* ws,
                        cudaStream_t s) {
   const int row = c->d_c + c->d_r;
-  const int S = append_splits(c), Kc = c->hidden / S;
   double* C = static_cast<double*>(ws);
   MLA_CUDA(cudaMemsetAsync(C, 0, sizeof(double) * (size_t)n * row, s));
-  GemmSimtArgs g1{x, W_DKV, C, n, c->d_c, Kc, S, c->hidden, 1, Kc, c->d_c, 1, (long long)Kc * c->d_c, row, 1, 0};
-  MLA_CUDA((gemm_simt<T, T, double, true>(g1, s)));
-  GemmSimtArgs g2{x, W_KR, C + c->d_c, n, c->d_r, Kc, S, c->hidden, 1, Kc, c->d_r, 1, (long long)Kc * c->d_r, row, 1, 0};
-  MLA_CUDA((gemm_simt<T, T, double, true>(g2, s)));
+  if (apf64::supports<T>(x, c->hidden, W_DKV, c->d_c, W_KR, c->d_r, c->d_c, c->d_r, c->hidden)) {
+    const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+    const int tiles = (row / apf64::BN) * ((n + apf64::BM - 1) / apf64::BM);
+    const int S = apf64::choose_splits(c->hidden, tiles, sms);
+    apf64::Args<T> a{static_cast<const T*>(x), c->hidden, static_cast<const T*>(W_DKV), c->d_c,
+                     static_cast<const T*>(W_KR), c->d_r, c->d_c, C, row, n, c->hidden / S};
+    MLA_CUDA(apf64::launch<T>(a, row, S, s));
+  } else {
+    const int S = append_splits(c), Kc = c->hidden / S;
+    GemmSimtArgs g1{x, W_DKV, C, n, c->d_c, Kc, S, c->hidden, 1, Kc, c->d_c, 1, (long long)Kc * c->d_c, row, 1, 0};
+    MLA_CUDA((gemm_simt<T, T, double, true>(g1, s)));
+    GemmSimtArgs g2{x, W_KR, C + c->d_c, n, c->d_r, Kc, S, c->hidden, 1, Kc, c->d_r, 1, (long long)Kc * c->d_r,
+                    row, 1, 0};
+    MLA_CUDA((gemm_simt<T, T, double, true>(g2, s)));
+  }
   const long long total = (long long)n * (c->d_c + c->d_r / 2);
   append_finish_kernel<T><<<grid_for(total), 256, 0, s>>>(
       C, 1, n, c->d_c, c->d_r, c->rope_theta, seq_idx, pos, static_cast<T*>(k->pool), k->block_table,
@@ -245,9 +262,9 @@ mla_status absorb_tc(const mla_config* c, const void* x, int n, const void* W_DQ
   if (c->q_lora > 0) MLA_TRY(wg::run(ps.dq, part, nullptr, cq_hi, cq_lo, s));
   MLA_TRY(wg::run(ps.uq, part, q_f, nullptr, nullptr, s));
   const int H = c->n_heads, nope = c->qk_nope;
-  const long long tot = (long long)n * H * (nope + c->d_r / 2);
-  query_split_bf16_kernel<<<grid_for(tot), 256, 0, s>>>(q_f, n, H, nope, c->d_r, c->rope_theta, pos, qn_hi, qn_lo,
-                                                        q_rope);
+  const dim3 qgrid(n, (H + kHeadGroup - 1) / kHeadGroup);
+  query_split_bf16_kernel<<<qgrid, 256, sizeof(double) * c->d_r, s>>>(q_f, n, H, nope, c->d_r, c->rope_theta, pos,
+                                                                     qn_hi, qn_lo, q_rope);
   note_launch();
   MLA_CUDA(cudaGetLastError());
   return wg::run(ps.uk, part, q_lat, nullptr, nullptr, s);
@@ -277,7 +294,7 @@ mla_status out_tc(const mla_config* c, const float* o_lat, int n, const void* W_
   bf16* ol = reinterpret_cast<bf16*>(base + w.ol);
   bf16* oh = reinterpret_cast<bf16*>(base + w.oh);
   const long long cnt = (long long)n * c->n_heads * c->d_c;
-  wg::split_bf16_kernel<<<grid_for(cnt), 256, 0, s>>>(o_lat, cnt, ol, nullptr);
+  wg::split_bf16_kernel<<<grid_for(cnt / 4), 256, 0, s>>>(o_lat, cnt, ol, nullptr);
   note_launch();
   MLA_CUDA(cudaGetLastError());
   const ProjSpecs ps = proj_specs(c, n, false, nullptr, nullptr, nullptr, W_UV, W_O, nullptr, nullptr, nullptr,
@@ -432,6 +449,7 @@ mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok, con
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cfg->dtype == MLA_BF16) {
     if (!proj_tc_supported(cfg)) return MLA_ERR_UNSUPPORTED;
+    if (!all_aligned16(x, W_DQ, W_UQ, W_UK, q_lat, q_rope, workspace)) return MLA_ERR_INVALID_ARG;
     if (ws_bytes < absorb_tc_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
     return absorb_tc(cfg, x, n_tok, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, workspace, s);
   }
@@ -455,6 +473,7 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
   MLA_TRY(check_cache(cache));
   if (cache->batch < batch) return MLA_ERR_INVALID_ARG;
   if (cfg->dtype == MLA_BF16 && !tcdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
+  if (cfg->dtype == MLA_BF16 && !all_aligned16(q_lat, q_rope, cache->pool, workspace)) return MLA_ERR_INVALID_ARG;
   const DecodeLayout L =
       decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers));
   if (ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
@@ -479,6 +498,7 @@ mla_status mla_combine(const mla_config* cfg, const void* workspace, size_t ws_b
   if (batch == 0) return MLA_OK;
   if (!workspace || !o_lat) return MLA_ERR_INVALID_ARG;
   if (ws_bytes < sizeof(DecodeHeader)) return MLA_ERR_WORKSPACE;
+  if (cfg->dtype == MLA_BF16 && !all_aligned16(workspace, o_lat)) return MLA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(batch * n_q, cfg->n_heads);
   combine_kernel<<<grid, 128, 0, s>>>(workspace, (long long)ws_bytes, batch, n_q, cfg->n_heads, cfg->d_c, o_lat);
@@ -501,6 +521,7 @@ mla_status mla_out_proj(const mla_config* cfg, const float* o_lat, int32_t n_tok
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cfg->dtype == MLA_BF16) {
     if (!proj_tc_supported(cfg)) return MLA_ERR_UNSUPPORTED;
+    if (!all_aligned16(o_lat, W_UV, W_O, y, workspace)) return MLA_ERR_INVALID_ARG;
     if (ws_bytes < out_tc_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
     return out_tc(cfg, o_lat, n_tok, W_UV, W_O, y, workspace, s);
   }

@@ -217,32 +217,54 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// out[i] = sum_s part[s][i] over `count` elements, written as fp32 and/or bf16
-// (hi) and/or the bf16 remainder (lo = value - hi).
-__global__ void reduce_splits_kernel(const float* __restrict__ part, int S, long long count, float* out_f32,
-                                     bf16* out_hi, bf16* out_lo) {
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
-       i += (long long)gridDim.x * blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < S; ++s) acc += part[(long long)s * count + i];
-    if (out_f32) out_f32[i] = acc;
-    if (out_hi) {
-      const bf16 h = __float2bfloat16_rn(acc);
-      out_hi[i] = h;
-      if (out_lo) out_lo[i] = __float2bfloat16_rn(acc - __bfloat162float(h));
+__device__ __forceinline__ void emit4(float4 v, long long i, float* out_f32, bf16* out_hi, bf16* out_lo) {
+  if (out_f32) *reinterpret_cast<float4*>(out_f32 + i) = v;
+  if (out_hi) {
+    const float a[4] = {v.x, v.y, v.z, v.w};
+    __align__(8) bf16 h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      h[e] = __float2bfloat16_rn(a[e]);
+      l[e] = __float2bfloat16_rn(a[e] - __bfloat162float(h[e]));
     }
+    *reinterpret_cast<uint2*>(out_hi + i) = *reinterpret_cast<const uint2*>(h);
+    if (out_lo) *reinterpret_cast<uint2*>(out_lo + i) = *reinterpret_cast<const uint2*>(l);
   }
 }
 
-// fp32 -> bf16 (hi) and optional remainder (lo).
-__global__ void split_bf16_kernel(const float* __restrict__ in, long long count, bf16* out_hi, bf16* out_lo) {
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
-       i += (long long)gridDim.x * blockDim.x) {
-    const float v = in[i];
-    const bf16 h = __float2bfloat16_rn(v);
-    out_hi[i] = h;
-    if (out_lo) out_lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+// out[i] = sum_s part[s][i] over `count` elements (a multiple of 4), summed in
+// split order, written as fp32 and/or bf16 (hi) and/or the bf16 remainder
+// (lo = value - hi).  Four elements per thread; the S loads of a group are
+// issued before the adds so they are in flight together.
+__global__ void reduce_splits_kernel(const float* __restrict__ part, int S, long long count, float* out_f32,
+                                     bf16* out_hi, bf16* out_lo) {
+  constexpr int kBatch = 8;
+  for (long long i = 4 * (blockIdx.x * (long long)blockDim.x + threadIdx.x); i < count;
+       i += 4LL * gridDim.x * blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < S; s0 += kBatch) {
+      float4 v[kBatch];
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b)
+        if (s0 + b < S) v[b] = __ldcs(reinterpret_cast<const float4*>(part + (long long)(s0 + b) * count + i));
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b)
+        if (s0 + b < S) {
+          acc.x += v[b].x;
+          acc.y += v[b].y;
+          acc.z += v[b].z;
+          acc.w += v[b].w;
+        }
+    }
+    emit4(acc, i, out_f32, out_hi, out_lo);
   }
+}
+
+// fp32 -> bf16 (hi) and optional remainder (lo); `count` a multiple of 4.
+__global__ void split_bf16_kernel(const float* __restrict__ in, long long count, bf16* out_hi, bf16* out_lo) {
+  for (long long i = 4 * (blockIdx.x * (long long)blockDim.x + threadIdx.x); i < count;
+       i += 4LL * gridDim.x * blockDim.x)
+    emit4(__ldg(reinterpret_cast<const float4*>(in + i)), i, nullptr, out_hi, out_lo);
 }
 
 }  // namespace wg
@@ -391,7 +413,7 @@ inline mla_status run(const Spec& s0, float* part, float* out_f32, bf16* out_hi,
   note_launch();
   if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
   const long long count = (long long)s.n_tok * s.G * s.F;
-  const int blocks = (int)std::min<long long>((count + 255) / 256, 4 * sms);
+  const int blocks = (int)std::min<long long>((count / 4 + 255) / 256, 8 * sms);
   reduce_splits_kernel<<<blocks, 256, 0, st>>>(part, S, count, out_f32, out_hi, out_lo);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;

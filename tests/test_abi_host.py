@@ -124,3 +124,28 @@ def test_decode_workspace_grows_with_workers_and_batch(lib):
 def test_status_strings(lib):
     for code in range(-6, 1):
         assert lib.mla_status_string(code)
+
+
+def test_unaligned_tensors_are_rejected_on_the_bf16_path(lib):
+    """TMA and 16-byte vector accesses need 16-byte aligned tensors; the bf16
+    entry points refuse an unaligned pointer before any launch."""
+    P = ctypes.byref
+    c = _cfg(hidden=7168, n_heads=128, d_c=512, d_r=64, qk_nope=128, v_head=128, q_lora=1536, dtype="bf16")
+    ok, bad = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10008)
+    need = lib.mla_absorb_q_workspace_size(P(c), 4)
+    assert need > 0
+    for i in range(7):
+        args = [ok] * 7
+        args[i] = bad          # x, W_DQ, W_UQ, W_UK, q_lat, q_rope, workspace (pos is int32, any alignment)
+        x, wdq, wuq, wuk, ql, qr, ws = args
+        assert lib.mla_absorb_q(P(c), x, 4, wdq, wuq, wuk, ok, ql, qr, ws, need, None) == abi.MLA_ERR_INVALID_ARG
+    need = lib.mla_out_proj_workspace_size(P(c), 4)
+    for i in range(5):
+        args = [ok] * 5
+        args[i] = bad
+        o, wuv, wo, y, ws = args
+        assert lib.mla_out_proj(P(c), o, 4, wuv, wo, y, ws, need, None) == abi.MLA_ERR_INVALID_ARG
+    cache = abi.MLACache(0x10008, 4, 0x3000, 1, 2)   # pool off the 16-byte grid
+    need = lib.mla_decode_workspace_size(P(c), 1, 1, 8)
+    assert lib.mla_decode(P(c), ok, ok, 1, 1, P(cache), ok, 8, ok, need, None) == abi.MLA_ERR_INVALID_ARG
+    assert lib.mla_combine(P(c), ok, need, 1, 1, bad, None) == abi.MLA_ERR_INVALID_ARG
