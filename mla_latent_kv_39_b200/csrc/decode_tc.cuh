@@ -34,7 +34,7 @@
 #pragma once
 
 #include "decode_plan.cuh"
-#include "decode_tc2.cuh"
+#include "decode_tc3.cuh"
 #include "sm100.cuh"
 
 namespace mla {
@@ -516,7 +516,7 @@ inline mla_status launch(const mla_config* c, const float* q_lat, const float* q
   Params p{q_lat, q_rope, k->block_table, seq_lens, k->max_blocks_per_seq, k->num_blocks, n_q,
            scale * 1.4426950408889634f, ws, L};
   const bool split = (c->flags & MLA_FLAG_SPLIT_QUERY) != 0;
-  const dim3 grid(2 * L.workers), block(kThreads), block2(tcdec2::kThreads);
+  const dim3 grid(2 * L.workers), block(kThreads);
   if (split) {
     if (set_smem_attr<true>() != MLA_OK) return MLA_ERR_CUDA;
     decode_tc_kernel<true><<<grid, block, smem_bytes<true>(), s>>>(map, p);
@@ -526,14 +526,14 @@ inline mla_status launch(const mla_config* c, const float* q_lat, const float* q
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
     const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
     if (!bit || !(done_mask.load(std::memory_order_acquire) & bit)) {
-      if (cudaFuncSetAttribute(tcdec2::decode_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)tcdec2::kSmemBytes) != cudaSuccess)
+      if (cudaFuncSetAttribute(tcdec3::decode_tc3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)tcdec3::kSmemBytes) != cudaSuccess)
         return MLA_ERR_CUDA;
       if (bit) done_mask.fetch_or(bit, std::memory_order_acq_rel);
     }
-    const tcdec2::Params p2{q_lat, q_rope, k->block_table, seq_lens, k->max_blocks_per_seq, k->num_blocks, n_q,
+    const tcdec3::Params p3{q_lat, q_rope, k->block_table, seq_lens, k->max_blocks_per_seq, k->num_blocks, n_q,
                             scale * 1.4426950408889634f, ws, L};
-    tcdec2::decode_tc2_kernel<<<grid, block2, tcdec2::kSmemBytes, s>>>(map, p2);
+    tcdec3::decode_tc3_kernel<<<grid, dim3(tcdec3::kThreads), tcdec3::kSmemBytes, s>>>(map, p3);
   }
   note_launch();
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
