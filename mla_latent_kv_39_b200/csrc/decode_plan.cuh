@@ -29,6 +29,7 @@ struct DecodeLayout {
   long long off_seg;           // int4  [max_segments] (v, blk_begin, blk_end, worker)
   long long off_lse;           // f32   [max_segments, H]        log2-sum-exp
   long long off_o;             // f32   [max_segments, H, d_c]   normalised partial output
+  long long off_qpack;         // bf16  [rows, H, d_c + d_r]     the query in bf16 (tensor-core path)
   long long total;
 };
 
@@ -38,7 +39,8 @@ struct DecodeHeader {
   DecodeLayout layout;
 };
 
-static inline DecodeLayout decode_layout(int batch, int n_q, int H, int d_c, int workers) {
+static inline DecodeLayout decode_layout(int batch, int n_q, int H, int d_c, int workers,
+                                         size_t qpack_row_bytes = 0) {
   DecodeLayout L{};
   const size_t rows = (size_t)batch * n_q;
   L.batch = batch;
@@ -55,6 +57,7 @@ static inline DecodeLayout decode_layout(int batch, int n_q, int H, int d_c, int
   L.off_seg = o;           o = align_up(o + sizeof(int4) * (size_t)L.max_segments, 256);
   L.off_lse = o;           o = align_up(o + sizeof(float) * (size_t)L.max_segments * H, 256);
   L.off_o = o;             o = align_up(o + sizeof(float) * (size_t)L.max_segments * H * d_c, 256);
+  L.off_qpack = o;         o = align_up(o + qpack_row_bytes * rows, 256);
   L.total = o;
   return L;
 }

@@ -491,6 +491,22 @@ inline mla_status pool_tensor_map(const mla_cache* k, CUtensorMap* map) {
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// The packed query (bf16 [rows * 128, 576], row stride 1152 B) read in boxes
+// of 128 heads x 64 values with the 128-byte swizzle: one box is one
+// shared-memory query slab of the decode.
+inline mla_status qpack_tensor_map(void* qpack, long long rows, CUtensorMap* map) {
+  EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return MLA_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)kRow, (cuuint64_t)rows * kH};
+  const cuuint64_t strides[1] = {(cuuint64_t)kRow * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kH};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qpack, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 template <bool kSplit>
 inline mla_status set_smem_attr() {
   static std::atomic<uint64_t> done_mask{0};  // one bit per device (devices 0..63)
@@ -531,9 +547,18 @@ inline mla_status launch(const mla_config* c, const float* q_lat, const float* q
         return MLA_ERR_CUDA;
       if (bit) done_mask.fetch_or(bit, std::memory_order_acq_rel);
     }
+    const long long rows = (long long)L.batch * L.n_q;
+    bf16* qpack = reinterpret_cast<bf16*>(static_cast<char*>(ws) + L.off_qpack);
+    CUtensorMap qmap;
+    const mla_status qs = qpack_tensor_map(qpack, rows, &qmap);
+    if (qs != MLA_OK) return qs;
+    const long long groups = rows * kH * (kRow / 8);
+    const int qblocks = (int)std::min<long long>((groups + 255) / 256, 16384);
+    tcdec3::q_pack_kernel<<<qblocks, 256, 0, s>>>(q_lat, q_rope, rows * kH, qpack);
+    note_launch();
     const tcdec3::Params p3{q_lat, q_rope, k->block_table, seq_lens, k->max_blocks_per_seq, k->num_blocks, n_q,
                             scale * 1.4426950408889634f, ws, L};
-    tcdec3::decode_tc3_kernel<<<grid, dim3(tcdec3::kThreads), tcdec3::kSmemBytes, s>>>(map, p3);
+    tcdec3::decode_tc3_kernel<<<grid, dim3(tcdec3::kThreads), tcdec3::kSmemBytes, s>>>(map, qmap, p3);
   }
   note_launch();
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;

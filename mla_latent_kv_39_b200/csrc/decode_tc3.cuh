@@ -65,7 +65,7 @@ struct Smem {
   uint8_t qs[kEarly][kQSlab];
   uint64_t early_full[2], val_full[2], early_free[2], val_free[2];
   uint64_t s_full[2], p_ready[2], pv_done[2];
-  uint64_t q_ready, s_fin, pv_fin;
+  uint64_t q_full, q_ready, s_fin, pv_fin;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -143,15 +143,11 @@ __device__ void producer(Smem& sm, const CUtensorMap* tmap, const Params& p, int
     const int phys = phys_block(p, segs, c, false);
     for (int s = 0; s < kRow / 64; ++s) prefetch_l2_2d(tmap, s * 64, phys * kBS);
   };
-  for (int i = 0; i < kPrefetch && ahead.valid(); ++i, ahead.next()) prefetch_page(ahead);
   int ne = 0, nv = 0;  // pages whose early / value loads were issued
+  int ai = 0;          // page index of `ahead`
   for (; cur.valid() && !aborted(sm); cur.next()) {
     const int k = ne, slot = k & 1;
     const uint32_t use = (uint32_t)k >> 1;
-    if (ahead.valid()) {
-      prefetch_page(ahead);
-      ahead.next();
-    }
     const int phys = phys_block(p, segs, cur, true);
     if (k >= 2 && !mbar_wait(&sm.early_free[slot], (use - 1) & 1, 40)) {
       set_abort(sm);
@@ -169,6 +165,10 @@ __device__ void producer(Smem& sm, const CUtensorMap* tmap, const Params& p, int
     for (int i = 0; i < kVal; ++i)
       tma_load_2d(sm.val[slot][i], tmap, val_slab(half, i) * 64, phys * kBS, &sm.val_full[slot]);
     ++nv;
+    // keep L2 warm kPrefetch pages ahead (after this page's own loads, so the
+    // first pages are not queued behind a burst of prefetches)
+    for (; ai <= k + kPrefetch && ahead.valid(); ++ai, ahead.next())
+      if (ai > k) prefetch_page(ahead);
   }
   // never leave a copy in flight into shared memory that is about to be released
   for (int kk = ne - 2 < 0 ? 0 : ne - 2; kk < ne; ++kk)
@@ -189,7 +189,7 @@ __device__ void score_issuer(Smem& sm, uint32_t tmem, const Params& p, int seg_b
   int k = 0, seg_i = 0;
   for (int si = seg_begin; si < seg_end; ++si, ++seg_i) {
     const int T = segs[si].z - segs[si].y;
-    if (!mbar_wait(&sm.q_ready, seg_i & 1, 50)) goto fail;
+    if (!mbar_wait(&sm.q_ready, seg_i & 1, 50) || !mbar_wait(&sm.q_full, seg_i & 1, 49)) goto fail;
     for (int i = 0; i < T; ++i) {
       const int kk = k + i, slot = kk & 1;
       const uint32_t use = (uint32_t)kk >> 1;
@@ -260,48 +260,64 @@ fail:
 // ---------------------------------------------------------------- softmax
 #define MLA_WARP_WAIT(expr) (__all_sync(0xffffffffu, (expr)))
 
-// Row r of query row v: this CTA's latent half -> TMEM (bf16 pairs); the
-// other latent half and the rotary query -> the five shared-memory slabs,
-// K-major with the 128-byte swizzle (16-byte chunk c of row r at c ^ (r & 7)).
-__device__ __forceinline__ void load_query(const Params& p, Smem& sm, int v, int r, int half, uint32_t taddr) {
-  const float* ql = p.q_lat + ((long long)v * kH + r) * kDc;
-#pragma unroll 1
-  for (int c = 0; c < 8; ++c) {  // 32 values -> 16 columns
-    const float4* src = reinterpret_cast<const float4*>(ql + 256 * half + c * 32);
-    uint32_t w[16];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 f = __ldg(src + i);
-      w[2 * i] = pack_bf16x2(f.x, f.y);
-      w[2 * i + 1] = pack_bf16x2(f.z, f.w);
-    }
-    tmem_st16(taddr + kTmemQ + c * 16, w);
+// The fp32 query rows packed once into bf16 rows [H][d_c + d_r] (q_lat then
+// q_rope) in the workspace, so the decode moves half the bytes and can load
+// the shared-memory part of a query with TMA.  Eight values per thread.
+__global__ void q_pack_kernel(const float* __restrict__ q_lat, const float* __restrict__ q_rope, long long heads,
+                              bf16* __restrict__ qpack) {
+  constexpr int kPer = kRow / 8;  // 72 groups of 8 per head row
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < heads * kPer;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long hrow = i / kPer;
+    const int g = (int)(i % kPer);
+    const float* src = g < kDc / 8 ? q_lat + hrow * kDc + g * 8 : q_rope + hrow * kDr + (g - kDc / 8) * 8;
+    const float4 a = __ldg(reinterpret_cast<const float4*>(src)), b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+    *reinterpret_cast<uint4*>(qpack + hrow * kRow + g * 8) =
+        make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
   }
+}
+
+// Query row v for this CTA: the five shared-memory slabs (the other latent
+// half and the rotary part, 128 heads x 64 values each) by TMA, counted on
+// q_full; this thread's head row of its own latent half (256 bf16, 512 B)
+// from the packed query into TMEM.
+__device__ __forceinline__ void load_query(const Params& p, Smem& sm, const CUtensorMap* qmap, int v, int r,
+                                           int half, int tid, uint32_t taddr) {
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&sm.q_full, kEarly * kQSlab);
+    for (int i = 0; i < kEarly; ++i) tma_load_2d(sm.qs[i], qmap, early_slab(half, i) * 64, v * kH, &sm.q_full);
+  }
+  const bf16* qpack = ws_at<bf16>(p.ws, p.L.off_qpack);
+  const uint4* src = reinterpret_cast<const uint4*>(qpack + ((long long)v * kH + r) * kRow + 256 * half);
 #pragma unroll 1
-  for (int e = 0; e < kEarly; ++e) {
-    const float* srcf = e < 4 ? ql + 256 * (1 - half) + 64 * e : p.q_rope + ((long long)v * kH + r) * kDr;
-    const float4* src = reinterpret_cast<const float4*>(srcf);
-    uint8_t* row = sm.qs[e] + r * 128;
+  for (int b = 0; b < 2; ++b) {  // 2 x 16 loads in flight, 64 columns each
+    uint4 w[16];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const float4 f0 = __ldg(src + 2 * c), f1 = __ldg(src + 2 * c + 1);
-      *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) * 16)) =
-          make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
-                     pack_bf16x2(f1.z, f1.w));
+    for (int i = 0; i < 16; ++i) w[i] = __ldg(src + b * 16 + i);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t x[16] = {w[4 * c].x,     w[4 * c].y,     w[4 * c].z,     w[4 * c].w,
+                              w[4 * c + 1].x, w[4 * c + 1].y, w[4 * c + 1].z, w[4 * c + 1].w,
+                              w[4 * c + 2].x, w[4 * c + 2].y, w[4 * c + 2].z, w[4 * c + 2].w,
+                              w[4 * c + 3].x, w[4 * c + 3].y, w[4 * c + 3].z, w[4 * c + 3].w};
+      tmem_st16(taddr + kTmemQ + b * 64 + c * 16, x);
     }
   }
 }
 
-// The next query row into L2, spread over the softmax threads (128-byte lines).
-__device__ __forceinline__ void prefetch_query(const Params& p, int v, int tid) {
-  const char* ql = reinterpret_cast<const char*>(p.q_lat + (long long)v * kH * kDc);
-  const char* qr = reinterpret_cast<const char*>(p.q_rope + (long long)v * kH * kDr);
-  for (int i = tid; i < kH * kDc * 4 / 128; i += 32 * kSoftmaxWarps) prefetch_line(ql + i * 128);
-  for (int i = tid; i < kH * kDr * 4 / 128; i += 32 * kSoftmaxWarps) prefetch_line(qr + i * 128);
+// The next query row into L2: its five slabs (tensor prefetch, one thread)
+// and this thread's TMEM part (four 128-byte lines).
+__device__ __forceinline__ void prefetch_query(const Params& p, const CUtensorMap* qmap, int v, int r, int half,
+                                               int tid) {
+  if (tid == 0)
+    for (int i = 0; i < kEarly; ++i) prefetch_l2_2d(qmap, early_slab(half, i) * 64, v * kH);
+  const bf16* qpack = ws_at<bf16>(p.ws, p.L.off_qpack);
+  const char* src = reinterpret_cast<const char*>(qpack + ((long long)v * kH + r) * kRow + 256 * half);
+  for (int i = 0; i < 4; ++i) prefetch_line(src + i * 128);
 }
 
-__device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_begin, int seg_end, int half,
-                             int warp, int lane) {
+__device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, const CUtensorMap* qmap, int seg_begin,
+                             int seg_end, int half, int warp, int lane) {
   const int4* segs = ws_at<int4>(p.ws, p.L.off_seg);
   const int qw = warp & 3;                                 // TMEM lane quarter
   const int r = qw * 32 + lane;                            // head row == TMEM lane
@@ -311,9 +327,8 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
   float* part_lse = ws_at<float>(p.ws, p.L.off_lse);
   if (seg_begin >= seg_end) return;
 
-  load_query(p, sm, segs[seg_begin].x, r, half, tl);
+  load_query(p, sm, qmap, segs[seg_begin].x, r, half, tid, tl);
   tmem_wait_st();
-  fence_proxy_async_smem();
   tc_fence_before();
   mbar_arrive(&sm.q_ready);
 
@@ -323,7 +338,7 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
     const int v = sg.x, b = v / p.n_q, jq = v % p.n_q;
     const int len_v = p.seq_lens[b] - p.n_q + jq + 1;
     const int T = sg.z - sg.y;
-    if (si + 1 < seg_end) prefetch_query(p, segs[si + 1].x, tid);
+    if (si + 1 < seg_end) prefetch_query(p, qmap, segs[si + 1].x, r, half, tid);
 
     float m_used = -INFINITY, l = 0.f;
     for (int i = 0; i < T; ++i) {
@@ -408,9 +423,8 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
     }
     // The scores of this segment are all done: the next query can replace this one.
     if (si + 1 < seg_end) {
-      load_query(p, sm, segs[si + 1].x, r, half, tl);
+      load_query(p, sm, qmap, segs[si + 1].x, r, half, tid, tl);
       tmem_wait_st();
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&sm.q_ready);
     }
@@ -443,6 +457,7 @@ fail:
 
 // ---------------------------------------------------------------- kernel
 __global__ void __launch_bounds__(kThreads, 1) decode_tc3_kernel(const __grid_constant__ CUtensorMap tmap,
+                                                                  const __grid_constant__ CUtensorMap qmap,
                                                                   const Params p) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -460,6 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc3_kernel(const __grid_co
       mbar_init(&sm.pv_done[b], 1);
     }
     mbar_init(&sm.q_ready, 32 * kSoftmaxWarps);
+    mbar_init(&sm.q_full, 1);
     mbar_init(&sm.s_fin, 1);
     mbar_init(&sm.pv_fin, 1);
     sm.abort_flag = 0;
@@ -469,7 +485,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc3_kernel(const __grid_co
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) prefetch_tensormap(&tmap);
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmap);
+    prefetch_tensormap(&qmap);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -489,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc3_kernel(const __grid_co
   } else if (warp == 2) {
     if (lane == 0) pv_issuer(sm, tmem, p, seg_begin, seg_end);
   } else {
-    softmax_role(sm, tmem, p, seg_begin, seg_end, half, warp, lane);
+    softmax_role(sm, tmem, p, &qmap, seg_begin, seg_end, half, warp, lane);
   }
 
   tc_fence_before();

@@ -312,6 +312,12 @@ int default_workers(const mla_config* c) {
   return std::max(1, 2 * sms);
 }
 
+// The tensor-core decode reads the query as bf16 rows [H, d_c + d_r] that a
+// first kernel packs from the fp32 inputs into the workspace.
+size_t qpack_row_bytes(const mla_config* c) {
+  return c->dtype == MLA_BF16 ? (size_t)c->n_heads * (c->d_c + c->d_r) * 2 : 0;
+}
+
 int resolve_workers(const mla_config* c, int max_workers) {
   return max_workers > 0 ? max_workers : default_workers(c);
 }
@@ -459,7 +465,9 @@ mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok, con
 
 size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t n_q, int32_t max_workers) {
   if (check_cfg(cfg) != MLA_OK || batch < 0 || n_q <= 0 || max_workers < 0) return 0;
-  return (size_t)decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers)).total;
+  return (size_t)decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers),
+                               qpack_row_bytes(cfg))
+      .total;
 }
 
 mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_rope, int32_t batch,
@@ -475,7 +483,7 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
   if (cfg->dtype == MLA_BF16 && !tcdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
   if (cfg->dtype == MLA_BF16 && !all_aligned16(q_lat, q_rope, cache->pool, workspace)) return MLA_ERR_INVALID_ARG;
   const DecodeLayout L =
-      decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers));
+      decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers), qpack_row_bytes(cfg));
   if (ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t plan_smem = sizeof(int) * ((size_t)batch * n_q + 1);
