@@ -9,7 +9,10 @@
 // "segment" - covers pages [blk_begin, blk_end) of one query row.  There are
 // at most workers + rows - 1 segments.  Each segment's decode writes, per
 // head, its output normalised over its own rows plus the log2-sum-exp of its
-// scaled scores; the combine merges the segments of a row.  The plan is
+// scaled scores; the combine merges the segments of a row.  The partial
+// outputs are stored head-minor ([segment][d][h]): the tensor-core decode
+// holds one head per TMEM lane, so a warp's 32 heads of one column form one
+// 128-byte store.  The plan is
 // computed on the device from seq_lens, so a decode step never waits on the
 // host.
 #pragma once
@@ -28,7 +31,7 @@ struct DecodeLayout {
   long long off_seq_nseg;      // int32 [rows]        number of segments of query row v
   long long off_seg;           // int4  [max_segments] (v, blk_begin, blk_end, worker)
   long long off_lse;           // f32   [max_segments, H]        log2-sum-exp
-  long long off_o;             // f32   [max_segments, H, d_c]   normalised partial output
+  long long off_o;             // f32   [max_segments, d_c, H]   normalised partial output (head-minor)
   long long off_qpack;         // bf16  [rows, H, d_c + d_r]     the query in bf16 (tensor-core path)
   long long total;
 };
@@ -197,58 +200,56 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   }
 }
 
-// o_lat[v, h, :] = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M) over the
-// segments of query row v.  Grid (query rows, heads), block over d_c.
+// o_lat[v, h, d] = sum_s 2^(lse_s,h - M_h) O_s[d, h] / sum_s 2^(lse_s,h - M_h)
+// over the segments s of query row v (M_h the largest lse_s,h).  Grid (query
+// rows, d_c / 32 column blocks), one thread per head (looping past 128 heads);
+// the 32-column x 128-head tile goes through shared memory, so the partial
+// outputs are read head-minor and o_lat is written column-minor, both in
+// whole 128-byte lines.
+constexpr int kCombDims = 32;
 __global__ void __launch_bounds__(128) combine_kernel(const void* ws, long long ws_bytes, int batch,
                                                       int n_q, int H, int d_c, float* __restrict__ o_lat) {
+  __shared__ float tile[kCombDims][129];
   const DecodeHeader* hd = ws_at<DecodeHeader>(ws, 0);
-  const int v = blockIdx.x, h = blockIdx.y;
-  float* out = o_lat + ((long long)v * H + h) * d_c;
-  if (hd->magic != kPlanMagic || hd->batch != batch || hd->n_q != n_q || hd->H != H ||
-      hd->d_c != d_c || hd->layout.total > ws_bytes) {
-    if (v == 0 && h == 0 && threadIdx.x == 0) report(MLA_ERR_WORKSPACE, 0, batch, n_q);
-    for (int d = threadIdx.x; d < d_c; d += blockDim.x) out[d] = 0.f;
-    return;
-  }
+  const int v = blockIdx.x, d0 = blockIdx.y * kCombDims, nd = min(kCombDims, d_c - d0);
+  const bool bad = hd->magic != kPlanMagic || hd->batch != batch || hd->n_q != n_q || hd->H != H ||
+                   hd->d_c != d_c || hd->layout.total > ws_bytes;
+  if (bad && v == 0 && blockIdx.y == 0 && threadIdx.x == 0) report(MLA_ERR_WORKSPACE, 0, batch, n_q);
   const DecodeLayout L = hd->layout;
-  const int first = ws_at<int>(ws, L.off_seq_first)[v];
-  const int n = ws_at<int>(ws, L.off_seq_nseg)[v];
+  const int first = bad ? 0 : ws_at<int>(ws, L.off_seq_first)[v];
+  const int n = bad ? 0 : ws_at<int>(ws, L.off_seq_nseg)[v];
   const float* lse = ws_at<float>(ws, L.off_lse);
   const float* part = ws_at<float>(ws, L.off_o);
-  float M = -INFINITY;
-  for (int s = 0; s < n; ++s) M = fmaxf(M, lse[(long long)(first + s) * H + h]);
-  if (n == 0 || M == -INFINITY) {
-    for (int d = threadIdx.x; d < d_c; d += blockDim.x) out[d] = 0.f;
-    return;
-  }
-  float Z = 0.f;
-  for (int s = 0; s < n; ++s) Z += exp2f(lse[(long long)(first + s) * H + h] - M);
-  const float invZ = 1.f / Z;
-  const bool vec = (d_c % 4 == 0) && ((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(part)) & 15u) == 0;
-  if (vec) {  // 16-byte loads of the partials, split weights evaluated once per split
-    for (int d = 4 * threadIdx.x; d < d_c; d += 4 * blockDim.x) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-      for (int s = 0; s < n; ++s) {
-        const long long r = (long long)(first + s) * H + h;
-        const float wgt = exp2f(lse[r] - M);
-        const float4 p4 = __ldcs(reinterpret_cast<const float4*>(part + r * d_c + d));
-        acc.x += wgt * p4.x;
-        acc.y += wgt * p4.y;
-        acc.z += wgt * p4.z;
-        acc.w += wgt * p4.w;
+  for (int h0 = 0; h0 < H; h0 += 128) {
+    const int h = h0 + threadIdx.x;
+    float acc[kCombDims];
+#pragma unroll
+    for (int i = 0; i < kCombDims; ++i) acc[i] = 0.f;
+    if (h < H && n > 0) {
+      float M = -INFINITY;
+      for (int s = 0; s < n; ++s) M = fmaxf(M, lse[(long long)(first + s) * H + h]);
+      if (M != -INFINITY) {
+        float Z = 0.f;
+        for (int s = 0; s < n; ++s) Z += exp2f(lse[(long long)(first + s) * H + h] - M);
+        const float invZ = 1.f / Z;
+        for (int s = 0; s < n; ++s) {
+          const long long seg = first + s;
+          const float w = exp2f(lse[seg * H + h] - M) * invZ;
+          const float* src = part + (seg * d_c + d0) * H + h;
+#pragma unroll
+          for (int i = 0; i < kCombDims; ++i)
+            if (i < nd) acc[i] = fmaf(w, __ldcs(src + (long long)i * H), acc[i]);
+        }
       }
-      *reinterpret_cast<float4*>(out + d) = make_float4(acc.x * invZ, acc.y * invZ, acc.z * invZ, acc.w * invZ);
     }
-    return;
-  }
-  for (int d = threadIdx.x; d < d_c; d += blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < n; ++s) {
-      const long long r = (long long)(first + s) * H + h;
-      acc += exp2f(lse[r] - M) * part[r * d_c + d];
+    __syncthreads();  // the previous head block's tile has been written out
+#pragma unroll
+    for (int i = 0; i < kCombDims; ++i) tile[i][threadIdx.x] = acc[i];
+    __syncthreads();
+    for (int e = threadIdx.x; e < 128 * kCombDims; e += 128) {
+      const int hh = e / kCombDims, i = e % kCombDims;
+      if (h0 + hh < H && i < nd) o_lat[((long long)v * H + h0 + hh) * d_c + d0 + i] = tile[i][hh];
     }
-    out[d] = acc * invZ;
   }
 }
 

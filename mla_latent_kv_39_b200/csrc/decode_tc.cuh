@@ -362,15 +362,14 @@ __device__ void softmax_role(Smem<kSplit>& sm, uint32_t tmem, const Params& p, i
       if (!MLA_WARP_WAIT(mbar_wait(&sm.pv_done, kl & 1, 33))) goto fail;
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      float4* out = reinterpret_cast<float4*>(part_o + ((long long)si * kH + r) * kDc + crank * 256);
+      // head-minor partial output: the warp's 32 heads of one column are one 128-byte line
+      float* out = part_o + ((long long)si * kDc + crank * 256) * kH + r;
       for (int ch = 0; ch < 8; ++ch) {
         uint32_t o[32];
         tmem_ld32(tl + kTmemO + ch * 32, o);
         tmem_wait_ld();
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
-          out[ch * 8 + t] = make_float4(__uint_as_float(o[4 * t]) * inv, __uint_as_float(o[4 * t + 1]) * inv,
-                                        __uint_as_float(o[4 * t + 2]) * inv, __uint_as_float(o[4 * t + 3]) * inv);
+        for (int t = 0; t < 32; ++t) out[(long long)(ch * 32 + t) * kH] = __uint_as_float(o[t]) * inv;
       }
       if (crank == 0) part_lse[(long long)si * kH + r] = l > 0.f ? m_used + log2f(l) : -INFINITY;
     }

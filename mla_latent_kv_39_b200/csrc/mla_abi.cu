@@ -508,7 +508,7 @@ mla_status mla_combine(const mla_config* cfg, const void* workspace, size_t ws_b
   if (ws_bytes < sizeof(DecodeHeader)) return MLA_ERR_WORKSPACE;
   if (cfg->dtype == MLA_BF16 && !all_aligned16(workspace, o_lat)) return MLA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  dim3 grid(batch * n_q, cfg->n_heads);
+  dim3 grid(batch * n_q, (cfg->d_c + kCombDims - 1) / kCombDims);
   combine_kernel<<<grid, 128, 0, s>>>(workspace, (long long)ws_bytes, batch, n_q, cfg->n_heads, cfg->d_c, o_lat);
   note_launch();
   return st(cudaGetLastError());
