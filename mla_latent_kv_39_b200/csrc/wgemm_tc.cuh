@@ -29,19 +29,29 @@ namespace wg {
 
 using namespace sm100;
 
-constexpr int kStages = 4;
+constexpr int kMaxStages = 12;
 constexpr int kABytes = 128 * 128;            // 128 features x 64 k, bf16
-constexpr int kStageBytes = 48 * 1024;        // A + up to 256 x 64 (or 2 x 128 x 64) of B
+constexpr int kRingBytes = 224 * 1024;        // stages of A + N x 64 (or 2 x N x 64) of B
 constexpr int kThreads = 192;
 
+// Stage size for an MMA N (1 KiB aligned for the swizzle atoms) and how many
+// fit the ring: 9 stages at N = 64, 4 at N = 256.
+__host__ __device__ constexpr int stage_bytes(int N, int split) {
+  return (kABytes + N * 128 * (split ? 2 : 1) + 1023) / 1024 * 1024;
+}
+__host__ __device__ constexpr int num_stages(int N, int split) {
+  return kRingBytes / stage_bytes(N, split) < kMaxStages ? kRingBytes / stage_bytes(N, split) : kMaxStages;
+}
+
 struct Smem {
-  uint8_t stage[kStages][kStageBytes];  // first member: 1024-byte aligned
-  uint64_t full[kStages], empty[kStages];
+  uint8_t ring[kRingBytes];  // first member: 1024-byte aligned
+  uint64_t full[kMaxStages], empty[kMaxStages];
   uint64_t acc_full[2], acc_empty[2];
   uint32_t tmem_base;
   int abort_flag;
 };
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory over the 227 KiB per-block limit");
 
 struct Params {
   int G, MT, KB, S;     // groups, 128-feature tiles per group, 64-k blocks per group, K splits
@@ -50,7 +60,10 @@ struct Params {
   int a_g_stride;       // MN-major: feature offset per group; K-major: k offset per group
   int split;            // B has a lo part
   int F;                // features per group
-  float* part;          // [S][n_tok][G][F]
+  float* part;          // [S][n_tok][G][F] (S > 1)
+  float* out_f32;       // with S == 1 the accumulator goes straight to the outputs [n_tok][G][F]
+  bf16* out_hi;
+  bf16* out_lo;
 };
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
@@ -82,9 +95,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int items = p.G * p.MT * p.S;
   const uint32_t b_bytes = (uint32_t)p.N * 128u;
   const uint32_t stage_tx = (uint32_t)kABytes + b_bytes * (p.split ? 2u : 1u);
+  const int nst = num_stages(p.N, p.split);
+  const uint32_t sbytes = (uint32_t)stage_bytes(p.N, p.split);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < nst; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
@@ -117,12 +132,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         int g, mt, kb0, kb1, s;
         item_coords(p, item, g, mt, kb0, kb1, s);
         for (int kb = kb0; kb < kb1; ++kb, ++k) {
-          const int st = k % kStages;
-          if (k >= kStages && !mbar_wait(&sm.empty[st], ((k / kStages) - 1) & 1, 70)) {
+          const int st = k % nst;
+          if (k >= nst && !mbar_wait(&sm.empty[st], ((k / nst) - 1) & 1, 70)) {
             set_abort(sm);
             goto producer_drain;
           }
-          uint8_t* a = sm.stage[st];
+          uint8_t* a = sm.ring + st * sbytes;
           uint8_t* b = a + kABytes;
           mbar_arrive_expect_tx(&sm.full[st], stage_tx);
           if (p.a_kmajor) {
@@ -136,8 +151,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     producer_drain:
-      for (int kk = k - kStages < 0 ? 0 : k - kStages; kk < k; ++kk)
-        mbar_wait(&sm.full[kk % kStages], (kk / kStages) & 1, 71);
+      for (int kk = k - nst < 0 ? 0 : k - nst; kk < k; ++kk)
+        mbar_wait(&sm.full[kk % nst], (kk / nst) & 1, 71);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -146,9 +161,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // A: MN-major -> 64-feature chunks 8 KiB apart (LBO), 8 k-rows 1 KiB apart
       // (SBO), K step j at +2 KiB * j; K-major -> rows 128 B apart, 8-row groups
       // 1 KiB apart (SBO), K step j at +32 B * j.  B: K-major like the latter.
-      const uint64_t a0 = p.a_kmajor ? smem_desc(smem_u32(sm.stage[0]), 16, 1024, kSwizzle128B)
-                                     : smem_desc(smem_u32(sm.stage[0]), kABytes / 2, 1024, kSwizzle128B);
-      const uint64_t b0 = smem_desc(smem_u32(sm.stage[0]) + kABytes, 16, 1024, kSwizzle128B);
+      const uint64_t a0 = p.a_kmajor ? smem_desc(smem_u32(sm.ring), 16, 1024, kSwizzle128B)
+                                     : smem_desc(smem_u32(sm.ring), kABytes / 2, 1024, kSwizzle128B);
+      const uint64_t b0 = smem_desc(smem_u32(sm.ring) + kABytes, 16, 1024, kSwizzle128B);
       int k = 0, j = 0;
       for (int item = blockIdx.x; item < items; item += gridDim.x, ++j) {
         int g, mt, kb0, kb1, s;
@@ -158,10 +173,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d = tmem + buf * 256;
         for (int kb = kb0; kb < kb1; ++kb, ++k) {
-          const int st = k % kStages;
-          if (!mbar_wait(&sm.full[st], (k / kStages) & 1, 73)) goto mma_fail;
+          const int st = k % nst;
+          if (!mbar_wait(&sm.full[st], (k / nst) & 1, 73)) goto mma_fail;
           tc_fence_after();
-          const uint32_t so = (uint32_t)(st * kStageBytes) >> 4;
+          const uint32_t so = (st * sbytes) >> 4;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const uint64_t ad = a0 + so + ((p.a_kmajor ? q * 32u : q * 2048u) >> 4);
@@ -194,14 +209,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const long long tstride = (long long)p.G * p.F;
-      float* out = p.part + (long long)s * p.n_tok * tstride + (long long)g * p.F + mt * 128 + f_local;
+      const long long col = (long long)g * p.F + mt * 128 + f_local;
+      float* out = p.part + (long long)s * p.n_tok * tstride + col;
       for (int c = 0; c < p.N; c += 32) {
         uint32_t v[32];
         tmem_ld32(tl + buf * 256 + c, v);
         tmem_wait_ld();
+        if (p.S > 1) {
 #pragma unroll
-        for (int t = 0; t < 32; ++t)
-          if (c + t < p.n_tok) out[(long long)(c + t) * tstride] = __uint_as_float(v[t]);
+          for (int t = 0; t < 32; ++t)
+            if (c + t < p.n_tok) out[(long long)(c + t) * tstride] = __uint_as_float(v[t]);
+        } else {  // one split: the step's outputs directly (a warp writes 32 consecutive features)
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            if (c + t >= p.n_tok) continue;
+            const float x = __uint_as_float(v[t]);
+            const long long o = (long long)(c + t) * tstride + col;
+            if (p.out_f32) p.out_f32[o] = x;
+            if (p.out_hi) {
+              const bf16 h = __float2bfloat16_rn(x);
+              p.out_hi[o] = h;
+              if (p.out_lo) p.out_lo[o] = __float2bfloat16_rn(x - __bfloat162float(h));
+            }
+          }
+        }
       }
       tc_fence_before();
       mbar_arrive(&sm.acc_empty[buf]);
@@ -315,20 +346,34 @@ inline bool spec_ok(const Spec& s) {
 // rows of one activation view (128 rows each of hi and lo).
 inline int max_chunk(const Spec& s) { return s.B_lo ? 128 : 256; }
 
-// K splits: enough work items to fill the SMs twice, while the partial sums
-// stay small next to the weights they come from.
+// K splits.  The grid has min(items, SMs) CTAs and CTA c takes items c,
+// c + grid, ...; the slowest CTA streams ceil(items / grid) items of about
+// KB / S 16 KiB weight blocks each.  With S > 1 every split also writes an
+// fp32 partial that a second kernel reads back (spread over all SMs, plus
+// that launch, counted as 128 KiB).  Pick the S with the fewest bytes on the
+// slowest SM, keeping the partials under a quarter of the weight bytes.
 inline int choose_splits(const Spec& s, int sms) {
   const int MT = s.F / 128, KB = s.Kg / 64;
   const long long base = (long long)s.G * MT;
-  int S = (int)std::max<long long>(1, std::min<long long>(KB, (2LL * sms + base - 1) / base));
   const double wbytes = 2.0 * s.G * (double)s.F * s.Kg;
-  const double out_bytes = 4.0 * s.G * (double)s.F * s.n_tok;
-  while (S > 1 && (S * out_bytes > 0.25 * wbytes || KB / S < 2)) --S;
-  return S;
+  const double out_bytes = 4.0 * s.G * (double)s.F * std::min(s.n_tok, max_chunk(s));
+  int best = 1;
+  double best_cost = -1.0;
+  for (int S = 1; S <= KB; ++S) {
+    if (S > 1 && S * out_bytes > 0.25 * wbytes) break;
+    const long long items = base * S, grid = std::min<long long>(items, sms);
+    double cost = (double)((items + grid - 1) / grid) * ((KB + S - 1) / S) * 16384.0;
+    if (S > 1) cost += 2.0 * S * out_bytes / sms + 131072.0;
+    if (best_cost < 0 || cost < best_cost) {
+      best = S;
+      best_cost = cost;
+    }
+  }
+  return best;
 }
 
 inline size_t partial_floats(const Spec& s, int S) {
-  return (size_t)S * std::min(s.n_tok, max_chunk(s)) * s.G * s.F;
+  return S > 1 ? (size_t)S * std::min(s.n_tok, max_chunk(s)) * s.G * s.F : 0;  // one split: no partials
 }
 
 inline int device_sms() {
@@ -407,11 +452,13 @@ inline mla_status run(const Spec& s0, float* part, float* out_f32, bf16* out_hi,
   mla_status ms = make_maps(s, N, &a, &bh, &bl);
   if (ms != MLA_OK) return ms;
   if ((ms = set_attr()) != MLA_OK) return ms;
-  Params p{s.G, s.F / 128, s.Kg / 64, S, s.n_tok, N, s.a_kmajor, s.a_g_stride, s.B_lo ? 1 : 0, s.F, part};
+  Params p{s.G, s.F / 128, s.Kg / 64, S, s.n_tok, N, s.a_kmajor, s.a_g_stride, s.B_lo ? 1 : 0, s.F, part,
+           out_f32, out_hi, out_lo};
   const int items = s.G * (s.F / 128) * S;
   wgemm_kernel<<<std::min(items, sms), kThreads, kSmemBytes, st>>>(a, bh, bl, p);
   note_launch();
   if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  if (S == 1) return MLA_OK;
   const long long count = (long long)s.n_tok * s.G * s.F;
   const int blocks = (int)std::min<long long>((count / 4 + 255) / 256, 8 * sms);
   reduce_splits_kernel<<<blocks, 256, 0, st>>>(part, S, count, out_f32, out_hi, out_lo);
