@@ -1,8 +1,10 @@
 // Exact latent projection of the cache append on the fp64 pipe.
 //
-// DeepSeek-V2 (arXiv 2405.04434), "Low-Rank Key-Value Joint Compression" and
-// "Decoupled Rotary Position Embedding": every new token stores c_KV = x W_DKV
-// and k_R = RoPE(x W_KR).  The cache is the bf16 rounding of the real-number
+// "Multi-head Latent Attention (MLA) Nedir?" (yapayzekasozluk.tr), section
+// "MLA nasıl çalışır?" (compression; decoupled RoPE), and "GQA, MQA ve MLA:
+// attention KV cache'i nasıl belirler" (LLMScale), section "Multi-head latent
+// attention (MLA)": every new token caches c_KV = x W_DKV and the small rotary
+// key k_R = RoPE(x W_KR).  The cache is the bf16 rounding of the real-number
 // product, so the sums are taken in fp64: a product of two bf16 (or fp32)
 // values is exact in fp64, only the fp64 additions round, and one final
 // rounding to bf16 then lands on the same value as rounding the exact sum

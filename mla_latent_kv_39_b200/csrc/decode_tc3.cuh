@@ -1,8 +1,8 @@
 // Latent-space split-KV decode on the sm_100 tensor cores.
 //
-// DeepSeek-V2 (arXiv 2405.04434), "Low-Rank Key-Value Joint Compression" and
-// "Decoupled Rotary Position Embedding", with W_UK absorbed into the query and
-// W_UV into the output: for every head h of query row v,
+// "MLA · latent KV, decoupled RoPE và matrix absorption" (openarchlab),
+// section 1 "Định nghĩa" and section 2 "Luồng": with W_UK absorbed into the
+// query and W_UV into the output side, for every head h of query row v
 //   s_t = q_lat[h] . c_t + q_R[h] . k_R,t          (t over the cached tokens)
 //   o_lat[h] = sum_t softmax(scale * s)_t c_t        (the latent output)
 // The split-KV plan hands every worker one contiguous run of pages (one or
