@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <utility>
 
 #include "mla.h"
 
@@ -26,6 +27,16 @@ __device__ __forceinline__ void report(int code, int a, int b, int c) {
     g_err[3] = c;
   }
 }
+
+// ------------------------------------------------------------ launch chaining
+// Kernels of a decode step are launched with programmatic stream
+// serialization: a kernel may start while the previous one in the stream is
+// finishing.  Each such kernel runs its prologue (barriers, TMEM, descriptor
+// prefetch), then pdl_wait() before it touches global memory the previous
+// kernels write or read, and pdl_trigger() to let the next one start.  Both
+// are no-ops for a normal launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ------------------------------------------------------------ storage types
 template <typename T> struct Store;
@@ -76,6 +87,26 @@ inline std::atomic<long long>& launch_counter() {
 static inline void note_launch(long long n = 1) { launch_counter().fetch_add(n, std::memory_order_relaxed); }
 
 static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Launch `kernel` so that it may overlap the tail of the previous kernel in
+// `s` (the kernel itself must call pdl_wait() before reading or writing
+// anything that kernel touches).
+template <typename... KArgs, typename... Args>
+static inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                         Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  note_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 static inline int elem_bytes(const mla_config* cfg) { return cfg->dtype == MLA_BF16 ? 2 : 4; }
 

@@ -129,6 +129,8 @@ constexpr int kPlanMaxRows = 49152;
 __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __restrict__ seq_lens,
                                                            int bs, int max_blocks, void* ws,
                                                            DecodeLayout L) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int P[];  // [rows + 1]
   int* wfirst = ws_at<int>(ws, L.off_worker_first);
   int* sfirst = ws_at<int>(ws, L.off_seq_first);
@@ -209,6 +211,8 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
 constexpr int kCombDims = 32;
 __global__ void __launch_bounds__(128) combine_kernel(const void* ws, long long ws_bytes, int batch,
                                                       int n_q, int H, int d_c, float* __restrict__ o_lat) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float tile[kCombDims][129];
   const DecodeHeader* hd = ws_at<DecodeHeader>(ws, 0);
   const int v = blockIdx.x, d0 = blockIdx.y * kCombDims, nd = min(kCombDims, d_c - d0);

@@ -553,11 +553,15 @@ inline mla_status launch(const mla_config* c, const float* q_lat, const float* q
     if (qs != MLA_OK) return qs;
     const long long groups = rows * kH * (kRow / 8);
     const int qblocks = (int)std::min<long long>((groups + 255) / 256, 16384);
-    tcdec3::q_pack_kernel<<<qblocks, 256, 0, s>>>(q_lat, q_rope, rows * kH, qpack);
-    note_launch();
+    if (launch_chained(tcdec3::q_pack_kernel, dim3(qblocks), dim3(256), 0, s, q_lat, q_rope, rows * kH, qpack) !=
+        cudaSuccess)
+      return MLA_ERR_CUDA;
     const tcdec3::Params p3{q_lat, q_rope, k->block_table, seq_lens, k->max_blocks_per_seq, k->num_blocks, n_q,
                             scale * 1.4426950408889634f, ws, L};
-    tcdec3::decode_tc3_kernel<<<grid, dim3(tcdec3::kThreads), tcdec3::kSmemBytes, s>>>(map, qmap, p3);
+    return launch_chained(tcdec3::decode_tc3_kernel, grid, dim3(tcdec3::kThreads), tcdec3::kSmemBytes, s, map, qmap,
+                          p3) == cudaSuccess
+               ? MLA_OK
+               : MLA_ERR_CUDA;
   }
   note_launch();
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;

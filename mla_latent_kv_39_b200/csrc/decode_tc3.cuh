@@ -265,6 +265,8 @@ fail:
 // the shared-memory part of a query with TMA.  Eight values per thread.
 __global__ void q_pack_kernel(const float* __restrict__ q_lat, const float* __restrict__ q_rope, long long heads,
                               bf16* __restrict__ qpack) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int kPer = kRow / 8;  // 72 groups of 8 per head row
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < heads * kPer;
        i += (long long)gridDim.x * blockDim.x) {
@@ -492,6 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc3_kernel(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  pdl_wait();  // the plan, the packed query and the appended rows come from the kernels before
+  pdl_trigger();
 
   int seg_begin = 0, seg_end = 0;
   if (worker < p.L.workers) {
@@ -500,12 +504,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc3_kernel(const __grid_co
     seg_end = wfirst[worker + 1];
   }
 
+  // The single-thread roles keep their warp's other lanes parked at a warp
+  // barrier (not at the CTA barrier below) while lane 0 works.
   if (warp == 0) {
     if (lane == 0) producer(sm, &tmap, p, seg_begin, seg_end, half);
+    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) score_issuer(sm, tmem, p, seg_begin, seg_end);
+    __syncwarp();
   } else if (warp == 2) {
     if (lane == 0) pv_issuer(sm, tmem, p, seg_begin, seg_end);
+    __syncwarp();
   } else {
     softmax_role(sm, tmem, p, &qmap, seg_begin, seg_end, half, warp, lane);
   }

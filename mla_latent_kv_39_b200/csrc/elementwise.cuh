@@ -55,6 +55,8 @@ __global__ void append_finish_kernel(const double* __restrict__ C, int splits, i
                                      const int32_t* __restrict__ pos, T* __restrict__ pool,
                                      const int32_t* __restrict__ block_table, int batch,
                                      int max_blocks, int num_blocks, int bs) {
+  pdl_wait();
+  pdl_trigger();
   const int per_tok = d_c + d_r / 2;
   const long long total = (long long)n_tok * per_tok;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
@@ -123,6 +125,8 @@ constexpr int kHeadGroup = 32;
 __global__ void query_split_bf16_kernel(const float* __restrict__ q, int n_tok, int H, int nope, int d_r,
                                         double theta, const int32_t* __restrict__ pos, bf16* __restrict__ q_nope,
                                         bf16* __restrict__ q_nope_lo, float* __restrict__ q_rope) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ double rot[];  // [d_r/2][cos, sin]
   const int t = blockIdx.x, half = d_r / 2, w = nope + d_r;
   for (int i = threadIdx.x; i < half; i += blockDim.x) {

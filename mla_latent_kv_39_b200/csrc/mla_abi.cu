@@ -101,11 +101,9 @@ mla_status append_impl(const mla_config* c, const void* x, int n, const void* W_
     MLA_CUDA((gemm_simt<T, T, double, true>(g2, s)));
   }
   const long long total = (long long)n * (c->d_c + c->d_r / 2);
-  append_finish_kernel<T><<<grid_for(total), 256, 0, s>>>(
-      C, 1, n, c->d_c, c->d_r, c->rope_theta, seq_idx, pos, static_cast<T*>(k->pool), k->block_table,
-      k->batch, k->max_blocks_per_seq, k->num_blocks, c->block_size);
-  note_launch();
-  return st(cudaGetLastError());
+  return st(launch_chained(append_finish_kernel<T>, dim3(grid_for(total)), dim3(256), 0, s, (const double*)C, 1, n,
+                            c->d_c, c->d_r, c->rope_theta, seq_idx, pos, static_cast<T*>(k->pool), k->block_table,
+                            k->batch, k->max_blocks_per_seq, k->num_blocks, c->block_size));
 }
 
 // ---------------------------------------------------------------- absorb
@@ -263,10 +261,8 @@ mla_status absorb_tc(const mla_config* c, const void* x, int n, const void* W_DQ
   MLA_TRY(wg::run(ps.uq, part, q_f, nullptr, nullptr, s));
   const int H = c->n_heads, nope = c->qk_nope;
   const dim3 qgrid(n, (H + kHeadGroup - 1) / kHeadGroup);
-  query_split_bf16_kernel<<<qgrid, 256, sizeof(double) * c->d_r, s>>>(q_f, n, H, nope, c->d_r, c->rope_theta, pos,
-                                                                     qn_hi, qn_lo, q_rope);
-  note_launch();
-  MLA_CUDA(cudaGetLastError());
+  MLA_CUDA(launch_chained(query_split_bf16_kernel, qgrid, dim3(256), sizeof(double) * c->d_r, s, (const float*)q_f, n, H,
+                          nope, c->d_r, c->rope_theta, pos, qn_hi, qn_lo, q_rope));
   return wg::run(ps.uk, part, q_lat, nullptr, nullptr, s);
 }
 
@@ -294,9 +290,8 @@ mla_status out_tc(const mla_config* c, const float* o_lat, int n, const void* W_
   bf16* ol = reinterpret_cast<bf16*>(base + w.ol);
   bf16* oh = reinterpret_cast<bf16*>(base + w.oh);
   const long long cnt = (long long)n * c->n_heads * c->d_c;
-  wg::split_bf16_kernel<<<grid_for(cnt / 4), 256, 0, s>>>(o_lat, cnt, ol, nullptr);
-  note_launch();
-  MLA_CUDA(cudaGetLastError());
+  MLA_CUDA(launch_chained(wg::split_bf16_kernel, dim3(grid_for(cnt / 4)), dim3(256), 0, s, o_lat, cnt, ol,
+                          (bf16*)nullptr));
   const ProjSpecs ps = proj_specs(c, n, false, nullptr, nullptr, nullptr, W_UV, W_O, nullptr, nullptr, nullptr,
                                   nullptr, nullptr, ol, oh);
   MLA_TRY(wg::run(ps.uv, part, nullptr, oh, nullptr, s));
@@ -491,9 +486,8 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
       cudaFuncSetAttribute(decode_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan_smem) !=
           cudaSuccess)
     return MLA_ERR_CUDA;
-  decode_plan_kernel<<<1, 1024, plan_smem, s>>>(seq_lens, cfg->block_size, cache->max_blocks_per_seq, workspace, L);
-  note_launch();
-  MLA_CUDA(cudaGetLastError());
+  MLA_CUDA(launch_chained(decode_plan_kernel, dim3(1), dim3(1024), plan_smem, s, seq_lens, cfg->block_size,
+                          cache->max_blocks_per_seq, workspace, L));
   if (cfg->dtype == MLA_BF16)
     return tcdec::launch(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, scale_of(cfg), s);
   return decode_simt_dispatch<float>(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, s);
@@ -509,9 +503,8 @@ mla_status mla_combine(const mla_config* cfg, const void* workspace, size_t ws_b
   if (cfg->dtype == MLA_BF16 && !all_aligned16(workspace, o_lat)) return MLA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   dim3 grid(batch * n_q, (cfg->d_c + kCombDims - 1) / kCombDims);
-  combine_kernel<<<grid, 128, 0, s>>>(workspace, (long long)ws_bytes, batch, n_q, cfg->n_heads, cfg->d_c, o_lat);
-  note_launch();
-  return st(cudaGetLastError());
+  return st(launch_chained(combine_kernel, grid, dim3(128), 0, s, (const void*)workspace, (long long)ws_bytes, batch,
+                            n_q, cfg->n_heads, cfg->d_c, o_lat));
 }
 
 size_t mla_out_proj_workspace_size(const mla_config* cfg, int32_t n_tok) {

@@ -73,14 +73,30 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// Work item -> (group, feature tile, K split).  Consecutive items (which run
+// on consecutive CTAs at about the same time) take neighbouring columns of the
+// weight matrix for the same K rows, so together they read whole DRAM pages
+// instead of 128-byte pieces of many: feature tiles then groups for
+// MN-major weights (columns g * F + 128 mt), groups first for K-major ones
+// (columns g * Kg + k).
 __device__ __forceinline__ void item_coords(const Params& p, int item, int& g, int& mt, int& kb0, int& kb1, int& s) {
-  const int per_g = p.MT * p.S;
-  g = item / per_g;
-  const int rem = item % per_g;
-  mt = rem / p.S;
-  s = rem % p.S;
+  const int tiles = p.G * p.MT;
+  s = item / tiles;
+  const int c = item % tiles;
+  if (p.a_kmajor) {
+    mt = c / p.G;
+    g = c % p.G;
+  } else {
+    g = c / p.MT;
+    mt = c % p.MT;
+  }
   kb0 = (int)((long long)s * p.KB / p.S);
   kb1 = (int)((long long)(s + 1) * p.KB / p.S);
+}
+
+__device__ __forceinline__ void prefetch_l2_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
 }
 
 __device__ __forceinline__ void set_abort(Smem& sm) { *(volatile int*)&sm.abort_flag = 1; }
@@ -123,6 +139,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  if (warp == 0 && lane == 0 && blockIdx.x < items) {
+    // The weights are not written by the kernels before this one: start
+    // pulling this CTA's first weight blocks into L2 while they finish.
+    int g, mt, kb0, kb1, s;
+    item_coords(p, blockIdx.x, g, mt, kb0, kb1, s);
+    for (int kb = kb0; kb < kb1 && kb < kb0 + nst; ++kb) {
+      if (p.a_kmajor) {
+        prefetch_l2_2d(&amap, g * p.a_g_stride + kb * 64, mt * 128);
+      } else {
+        prefetch_l2_2d(&amap, g * p.a_g_stride + mt * 128, kb * 64);
+        prefetch_l2_2d(&amap, g * p.a_g_stride + mt * 128 + 64, kb * 64);
+      }
+    }
+  }
+  pdl_wait();  // activations and output buffers belong to the kernels before
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -269,6 +301,8 @@ __device__ __forceinline__ void emit4(float4 v, long long i, float* out_f32, bf1
 // issued before the adds so they are in flight together.
 __global__ void reduce_splits_kernel(const float* __restrict__ part, int S, long long count, float* out_f32,
                                      bf16* out_hi, bf16* out_lo) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int kBatch = 8;
   for (long long i = 4 * (blockIdx.x * (long long)blockDim.x + threadIdx.x); i < count;
        i += 4LL * gridDim.x * blockDim.x) {
@@ -293,6 +327,8 @@ __global__ void reduce_splits_kernel(const float* __restrict__ part, int S, long
 
 // fp32 -> bf16 (hi) and optional remainder (lo); `count` a multiple of 4.
 __global__ void split_bf16_kernel(const float* __restrict__ in, long long count, bf16* out_hi, bf16* out_lo) {
+  pdl_wait();
+  pdl_trigger();
   for (long long i = 4 * (blockIdx.x * (long long)blockDim.x + threadIdx.x); i < count;
        i += 4LL * gridDim.x * blockDim.x)
     emit4(__ldg(reinterpret_cast<const float4*>(in + i)), i, nullptr, out_hi, out_lo);
@@ -455,15 +491,16 @@ inline mla_status run(const Spec& s0, float* part, float* out_f32, bf16* out_hi,
   Params p{s.G, s.F / 128, s.Kg / 64, S, s.n_tok, N, s.a_kmajor, s.a_g_stride, s.B_lo ? 1 : 0, s.F, part,
            out_f32, out_hi, out_lo};
   const int items = s.G * (s.F / 128) * S;
-  wgemm_kernel<<<std::min(items, sms), kThreads, kSmemBytes, st>>>(a, bh, bl, p);
-  note_launch();
-  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  if (launch_chained(wgemm_kernel, dim3(std::min(items, sms)), dim3(kThreads), kSmemBytes, st, a, bh, bl, p) !=
+      cudaSuccess)
+    return MLA_ERR_CUDA;
   if (S == 1) return MLA_OK;
   const long long count = (long long)s.n_tok * s.G * s.F;
   const int blocks = (int)std::min<long long>((count / 4 + 255) / 256, 8 * sms);
-  reduce_splits_kernel<<<blocks, 256, 0, st>>>(part, S, count, out_f32, out_hi, out_lo);
-  note_launch();
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return launch_chained(reduce_splits_kernel, dim3(blocks), dim3(256), 0, st, (const float*)part, S, count, out_f32,
+                        out_hi, out_lo) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
 }
 
 inline size_t run_partial_bytes(const Spec& s0) {
