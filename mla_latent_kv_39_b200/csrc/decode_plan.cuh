@@ -4,9 +4,10 @@
 // Row v sees the cache rows 0 .. len_v - 1 of sequence b, with
 // len_v = seq_lens[b] - n_q + j + 1 (causal, its own row included), i.e.
 // ceil(len_v / block) pages.  The pages of all query rows, laid end to end,
-// are cut into `workers` contiguous, equally sized ranges (+-1 page); where a
-// range crosses a row boundary it is cut again, so every piece - a
-// "segment" - covers pages [blk_begin, blk_end) of one query row.  There are
+// are cut into `workers` contiguous ranges of about equal cost (pages plus a
+// fixed charge per row for the segment's setup); where a range crosses a row
+// boundary it is cut again, so every piece - a "segment" - covers pages
+// [blk_begin, blk_end) of one query row.  There are
 // at most workers + rows - 1 segments.  Each segment's decode writes, per
 // head, its output normalised over its own rows plus the log2-sum-exp of its
 // scaled scores; the combine merges the segments of a row.  The partial
@@ -125,6 +126,7 @@ __device__ __forceinline__ int seq_of_page(const int* P, int rows, long long g) 
 // Page prefix of the query rows lives in shared memory (the searches below
 // are chains of dependent loads); one CTA computes the whole plan.
 constexpr int kPlanMaxRows = 49152;
+constexpr int kSegCost = 10;  // per-segment overhead of the decode, in quarter pages
 
 __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __restrict__ seq_lens,
                                                            int bs, int max_blocks, void* ws,
@@ -150,9 +152,25 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   };
   const int NB = block_scan_exclusive(pages_of, P, rows);
 
+  // Workers get equal shares of cost, not of pages: a segment costs a
+  // query reload and an epilogue on top of its pages (about kSegCost / 4
+  // pages), so every row is charged that much once.  Cost positions are in
+  // quarter pages; row v occupies [Pc(v), Pc(v + 1)) with Pc(v) = 4 P[v] +
+  // kSegCost v, its first kSegCost quarters being the overhead.
+  const long long NC = 4LL * NB + (long long)kSegCost * rows;
+  auto page_at = [&](long long x) -> long long {
+    int lo = 0, hi = rows - 1;  // largest v with Pc(v) <= x
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (4LL * P[mid] + (long long)kSegCost * mid <= x) lo = mid; else hi = mid - 1;
+    }
+    const long long o = x - (4LL * P[lo] + (long long)kSegCost * lo) - kSegCost;
+    const long long pages = P[lo + 1] - P[lo];
+    return P[lo] + (o <= 0 ? 0 : (o / 4 < pages ? o / 4 : pages));
+  };
   auto range_of = [&](int w, long long& s, long long& e) {
-    s = (long long)w * NB / W;
-    e = (long long)(w + 1) * NB / W;
+    s = page_at((long long)w * NC / W);
+    e = page_at((long long)(w + 1) * NC / W);
   };
   auto segs_of = [&](int w) -> int {
     long long s, e;
