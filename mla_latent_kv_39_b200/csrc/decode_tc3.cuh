@@ -165,10 +165,14 @@ __device__ void producer(Smem& sm, const CUtensorMap* tmap, const Params& p, int
     for (int i = 0; i < kVal; ++i)
       tma_load_2d(sm.val[slot][i], tmap, val_slab(half, i) * 64, phys * kBS, &sm.val_full[slot]);
     ++nv;
-    // keep L2 warm kPrefetch pages ahead (after this page's own loads, so the
-    // first pages are not queued behind a burst of prefetches)
-    for (; ai <= k + kPrefetch && ahead.valid(); ++ai, ahead.next())
-      if (ai > k) prefetch_page(ahead);
+    // keep L2 warm kPrefetch pages ahead, growing the window by at most two
+    // pages per loaded page (a start-up burst of prefetches from every CTA
+    // would delay everyone's first pages)
+    for (int n = 0; n < 2 && ai <= k + kPrefetch && ahead.valid(); ++ai, ahead.next())
+      if (ai > k) {
+        prefetch_page(ahead);
+        ++n;
+      }
   }
   // never leave a copy in flight into shared memory that is about to be released
   for (int kk = ne - 2 < 0 ? 0 : ne - 2; kk < ne; ++kk)
