@@ -128,11 +128,10 @@ __device__ __forceinline__ int seq_of_page(const int* P, int rows, long long g) 
 constexpr int kPlanMaxRows = 49152;
 constexpr int kSegCost = 10;  // per-segment overhead of the decode, in quarter pages
 
-__global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __restrict__ seq_lens,
-                                                           int bs, int max_blocks, void* ws,
-                                                           DecodeLayout L) {
-  pdl_wait();
-  pdl_trigger();
+// The plan, computed by one CTA of 1024 threads with (rows + 1) ints of
+// dynamic shared memory.
+__device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, int bs, int max_blocks, void* ws,
+                                          const DecodeLayout& L) {
   extern __shared__ int P[];  // [rows + 1]
   int* wfirst = ws_at<int>(ws, L.off_worker_first);
   int* sfirst = ws_at<int>(ws, L.off_seq_first);
@@ -218,6 +217,13 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
     h->num_segments = nsegs;
     h->layout = L;
   }
+}
+
+__global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __restrict__ seq_lens, int bs,
+                                                           int max_blocks, void* ws, DecodeLayout L) {
+  pdl_wait();
+  pdl_trigger();
+  plan_body(seq_lens, bs, max_blocks, ws, L);
 }
 
 // o_lat[v, h, d] = sum_s 2^(lse_s,h - M_h) O_s[d, h] / sum_s 2^(lse_s,h - M_h)

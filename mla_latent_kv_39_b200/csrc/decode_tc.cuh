@@ -520,9 +520,12 @@ inline mla_status set_smem_attr() {
   return MLA_OK;
 }
 
+// Launch the tensor-core decode.  With `with_plan` (the non-split path) the
+// split plan is computed in the same launch as the query packing; otherwise
+// the caller has launched the plan already.
 inline mla_status launch(const mla_config* c, const float* q_lat, const float* q_rope, int n_q,
                          const mla_cache* k, const int32_t* seq_lens, void* ws, const DecodeLayout& L,
-                         float scale, cudaStream_t s) {
+                         float scale, cudaStream_t s, size_t plan_smem) {
   if (((uintptr_t)k->pool & 15u) != 0 || ((uintptr_t)q_lat & 15u) != 0 || ((uintptr_t)q_rope & 15u) != 0)
     return MLA_ERR_INVALID_ARG;
   CUtensorMap map;
@@ -552,9 +555,13 @@ inline mla_status launch(const mla_config* c, const float* q_lat, const float* q
     const mla_status qs = qpack_tensor_map(qpack, rows, &qmap);
     if (qs != MLA_OK) return qs;
     const long long groups = rows * kH * (kRow / 8);
-    const int qblocks = (int)std::min<long long>((groups + 255) / 256, 16384);
-    if (launch_chained(tcdec3::q_pack_kernel, dim3(qblocks), dim3(256), 0, s, q_lat, q_rope, rows * kH, qpack) !=
-        cudaSuccess)
+    const int qblocks = (int)std::min<long long>((groups + 1023) / 1024, 4096);
+    if (plan_smem > 48 * 1024 && cudaFuncSetAttribute(tcdec3::plan_pack_kernel,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      (int)plan_smem) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    if (launch_chained(tcdec3::plan_pack_kernel, dim3(1 + qblocks), dim3(1024), plan_smem, s, seq_lens, c->block_size,
+                       k->max_blocks_per_seq, ws, L, q_lat, q_rope, rows * kH, qpack) != cudaSuccess)
       return MLA_ERR_CUDA;
     const tcdec3::Params p3{q_lat, q_rope, k->block_table, seq_lens, k->max_blocks_per_seq, k->num_blocks, n_q,
                             scale * 1.4426950408889634f, ws, L};

@@ -264,16 +264,24 @@ fail:
 // ---------------------------------------------------------------- softmax
 #define MLA_WARP_WAIT(expr) (__all_sync(0xffffffffu, (expr)))
 
-// The fp32 query rows packed once into bf16 rows [H][d_c + d_r] (q_lat then
-// q_rope) in the workspace, so the decode moves half the bytes and can load
-// the shared-memory part of a query with TMA.  Eight values per thread.
-__global__ void q_pack_kernel(const float* __restrict__ q_lat, const float* __restrict__ q_rope, long long heads,
-                              bf16* __restrict__ qpack) {
+// The fp32 query rows are packed once into bf16 rows [H][d_c + d_r] (q_lat
+// then q_rope) in the workspace, so the decode moves half the bytes and can
+// load the shared-memory part of a query with TMA.  Eight values per thread.
+// The split plan (block 0) and the query packing (the other blocks) in one
+// launch; both only read the step's inputs.
+__global__ void __launch_bounds__(1024) plan_pack_kernel(const int32_t* __restrict__ seq_lens, int bs, int max_blocks,
+                                                         void* ws, DecodeLayout L, const float* __restrict__ q_lat,
+                                                         const float* __restrict__ q_rope, long long heads,
+                                                         bf16* __restrict__ qpack) {
   pdl_wait();
   pdl_trigger();
-  constexpr int kPer = kRow / 8;  // 72 groups of 8 per head row
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < heads * kPer;
-       i += (long long)gridDim.x * blockDim.x) {
+  if (blockIdx.x == 0) {
+    plan_body(seq_lens, bs, max_blocks, ws, L);
+    return;
+  }
+  constexpr int kPer = kRow / 8;
+  for (long long i = (blockIdx.x - 1) * (long long)blockDim.x + threadIdx.x; i < heads * kPer;
+       i += (long long)(gridDim.x - 1) * blockDim.x) {
     const long long hrow = i / kPer;
     const int g = (int)(i % kPer);
     const float* src = g < kDc / 8 ? q_lat + hrow * kDc + g * 8 : q_rope + hrow * kDr + (g - kDc / 8) * 8;

@@ -482,14 +482,17 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
   if (ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t plan_smem = sizeof(int) * ((size_t)batch * n_q + 1);
-  if (plan_smem > 48 * 1024 &&
-      cudaFuncSetAttribute(decode_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan_smem) !=
-          cudaSuccess)
-    return MLA_ERR_CUDA;
-  MLA_CUDA(launch_chained(decode_plan_kernel, dim3(1), dim3(1024), plan_smem, s, seq_lens, cfg->block_size,
-                          cache->max_blocks_per_seq, workspace, L));
+  const bool fused_plan = cfg->dtype == MLA_BF16 && !(cfg->flags & MLA_FLAG_SPLIT_QUERY);
+  if (!fused_plan) {
+    if (plan_smem > 48 * 1024 &&
+        cudaFuncSetAttribute(decode_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan_smem) !=
+            cudaSuccess)
+      return MLA_ERR_CUDA;
+    MLA_CUDA(launch_chained(decode_plan_kernel, dim3(1), dim3(1024), plan_smem, s, seq_lens, cfg->block_size,
+                            cache->max_blocks_per_seq, workspace, L));
+  }
   if (cfg->dtype == MLA_BF16)
-    return tcdec::launch(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, scale_of(cfg), s);
+    return tcdec::launch(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, scale_of(cfg), s, plan_smem);
   return decode_simt_dispatch<float>(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, s);
 }
 
