@@ -121,7 +121,7 @@ __global__ void query_split_kernel(const float* __restrict__ q, int n_tok, int H
 // fp64).  One block per (token, group of kHeadGroup heads): the token's d_r/2
 // rotation angles are evaluated once into shared memory and shared by every
 // head.  Needs even nope and d_r (pairs are read and written together).
-constexpr int kHeadGroup = 32;
+constexpr int kHeadGroup = 8;
 __global__ void query_split_bf16_kernel(const float* __restrict__ q, int n_tok, int H, int nope, int d_r,
                                         double theta, const int32_t* __restrict__ pos, bf16* __restrict__ q_nope,
                                         bf16* __restrict__ q_nope_lo, float* __restrict__ q_rope) {
