@@ -26,6 +26,11 @@
  *    except where an argument says otherwise.  `stream` is a cudaStream_t
  *    (NULL = legacy default stream).  Every call is asynchronous on `stream`
  *    and never synchronises, except mla_get_device_error.
+ *  - Kernels are launched with programmatic stream serialization: one may
+ *    begin its set-up (barriers, tensor-memory allocation, warming L2 with
+ *    weights) while the previous kernel in the stream is finishing, but it
+ *    reads or writes no argument or workspace before that kernel completes,
+ *    so stream order is kept exactly.
  *  - Ownership: the caller owns every buffer, including the workspaces whose
  *    sizes the *_workspace_size queries return.  The library allocates no
  *    device memory.  Its only device state is one error word per device
