@@ -269,8 +269,7 @@ def run_ours(args):
     def one_step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        layer.append(x, seq_idx, pos)
-        layer.queries(x, pos)
+        layer.append_and_queries(x, seq_idx, pos)
         if ev is not None:
             ev[1].record(stream)
         layer.decode(seq_lens)

@@ -31,11 +31,13 @@ using namespace sm100;
 
 constexpr int kMaxStages = 12;
 constexpr int kABytes = 128 * 128;            // 128 features x 64 k, bf16
-constexpr int kRingBytes = 224 * 1024;        // stages of A + N x 64 (or 2 x N x 64) of B
+// 144 KiB: 6 stages at N = 64 stream as fast as 12, and leave room on each SM
+// for the append kernel, which runs beside the query projections.
+constexpr int kRingBytes = 144 * 1024;        // stages of A + N x 64 (or 2 x N x 64) of B
 constexpr int kThreads = 192;
 
 // Stage size for an MMA N (1 KiB aligned for the swizzle atoms) and how many
-// fit the ring: 9 stages at N = 64, 4 at N = 256.
+// fit the ring: 6 stages at N = 64, 3 at N = 256.
 __host__ __device__ constexpr int stage_bytes(int N, int split) {
   return (kABytes + N * 128 * (split ? 2 : 1) + 1023) / 1024 * 1024;
 }

@@ -34,6 +34,11 @@ class DecodeLayer:
         self.ws_gemm = torch.empty(max(gemm_ws, 256), dtype=torch.uint8, device=dev)
         self.ws_decode = torch.empty(abi.mla_decode_workspace_size(cfg, batch, n_q, max_workers),
                                      dtype=torch.uint8, device=dev)
+        # The step's append runs on a second stream beside the query projections
+        # (fp64 work next to weight streaming), with a workspace of its own.
+        self.side = torch.cuda.Stream(device=dev)
+        self.ws_append = torch.empty(max(abi.mla_cache_append_workspace_size(cfg, n), 256), dtype=torch.uint8,
+                                     device=dev)
 
     def _gemm_ws(self, n: int) -> torch.Tensor:
         need = max(abi.mla_cache_append_workspace_size(self.cfg, n), abi.mla_absorb_q_workspace_size(self.cfg, n),
@@ -53,6 +58,27 @@ class DecodeLayer:
         abi.mla_absorb_q(self.cfg, x, W_DQ, W_UQ, self.W["W_UK"], pos, self.q_lat, self.q_rope,
                          self.ws_gemm, stream)
 
+    def append_and_queries(self, x, seq_idx, pos, stream=None):
+        """The append and the query projections of one step, overlapped: the
+        projections go first on ``stream`` (so their CTAs are placed first), the
+        append on a side stream; ``stream`` waits for both before returning."""
+        main = stream or torch.cuda.current_stream()
+        ready = torch.cuda.Event()
+        ready.record(main)
+        self.queries(x, pos, main)
+        self.side.wait_event(ready)
+        need = abi.mla_cache_append_workspace_size(self.cfg, x.shape[0])
+        if need > self.ws_append.numel():
+            self.ws_append = torch.empty(need, dtype=torch.uint8, device=self.ws_append.device)
+        abi.mla_cache_append(self.cfg, x, self.W["W_DKV"], self.W["W_KR"], seq_idx, pos, self.cache,
+                             self.ws_append, self.side)
+        done = torch.cuda.Event()
+        done.record(self.side)
+        main.wait_event(done)
+        # keep the inputs alive until the side stream has used them
+        for t in (x, seq_idx, pos):
+            t.record_stream(self.side)
+
     def decode(self, seq_lens, stream=None):
         abi.mla_decode(self.cfg, self.q_lat, self.q_rope, self.batch, self.n_q, self.cache, seq_lens,
                        self.ws_decode, self.max_workers, stream)
@@ -69,8 +95,7 @@ class DecodeLayer:
 
     def step(self, x, seq_idx, pos, seq_lens, stream=None) -> torch.Tensor:
         """Device-resident step: returns ``y`` ``[batch * n_q, hidden]`` (a reused buffer)."""
-        self.append(x, seq_idx, pos, stream)
-        self.queries(x, pos, stream)
+        self.append_and_queries(x, seq_idx, pos, stream)
         self.attend(seq_lens, stream)
         self.project(stream)
         return self.y
