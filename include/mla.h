@@ -192,10 +192,11 @@ mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok,
  * position p = seq_lens[b] - n_q + j) and head h:
  *   s_u = (q_lat[t,h] . c_u + q_rope[t,h] . kR_u) * scale   for rows u <= p
  *   o_lat[t,h] = sum_u softmax(s)_u c_u
- * The rows of every sequence are split into contiguous page ranges, one per
- * scheduled worker; each range writes an unnormalised-free partial
- * (softmax-normalised over its rows) and its log2-sum-exp into `workspace`;
- * mla_combine merges them.
+ * The pages of all query rows are split into contiguous ranges of about
+ * equal cost, one per scheduled worker (the plan is computed on the device
+ * from seq_lens); each piece writes its output normalised over its own rows
+ * and its log2-sum-exp into `workspace`, and mla_combine merges them.  On the
+ * bf16 path the workspace also holds a packed bf16 copy of the query.
  *   q_lat float32 [batch n_q, H, d_c], q_rope float32 [batch n_q, H, d_r]:
  *            from mla_absorb_q (row v = b n_q + j)
  *   seq_lens int32 [batch]: rows of each sequence INCLUDING the n_q new rows
