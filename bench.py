@@ -83,7 +83,7 @@ def measured_peaks():
 
 # The sources the decode kernel is built from: a recorded DRAM traffic figure
 # is only reported while none of them has changed since it was measured.
-DECODE_SOURCES = ("common.cuh", "sm100.cuh", "decode_plan.cuh", "decode_tc.cuh", "decode_tc3.cuh")
+DECODE_SOURCES = ("common.cuh", "sm100.cuh", "decode_plan.cuh", "decode_pair.cuh")
 
 
 def kernel_source_hash() -> str:

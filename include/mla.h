@@ -246,6 +246,16 @@ mla_status mla_out_proj(const mla_config* cfg, const float* o_lat, int32_t n_tok
  * current device since the last call (MLA_OK if none) and clears it.
  * detail (may be NULL) receives 3 ints describing the failing item. */
 mla_status mla_get_device_error(void* stream, int32_t* detail);
+/* Check of the bounded-wait path (not on the pages; a test of this library's
+ * hang protection).  Every wait of the tensor-core kernels on a barrier gives
+ * up after a time limit (2 s in the decode), records MLA_ERR_TIMEOUT in the
+ * device error word and lets the kernel return, so a lost arrival surfaces
+ * as an error instead of a hung GPU.  This call launches a one-warp kernel
+ * that waits on a barrier whose second arrival never comes, with the given
+ * limit (1 ns .. 10 s); after it, mla_get_device_error returns
+ * MLA_ERR_TIMEOUT (detail[0] = 1) and the stream stays usable.
+ * Returns MLA_ERR_INVALID_ARG for a limit out of range. */
+mla_status mla_check_wait_timeout(int64_t limit_ns, void* stream);
 /* Static description of a status code. */
 const char* mla_status_string(mla_status status);
 /* MLA_ABI_VERSION of the loaded library. */

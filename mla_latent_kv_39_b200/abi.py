@@ -69,6 +69,7 @@ SIGNATURES = {
     "mla_out_proj_workspace_size": (_sz, [_P_CFG, _i32]),
     "mla_out_proj": (_i32, [_P_CFG, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mla_get_device_error": (_i32, [_vp, ctypes.POINTER(_i32)]),
+    "mla_check_wait_timeout": (_i32, [ctypes.c_int64, _vp]),
 }
 
 
@@ -291,6 +292,11 @@ def mla_get_device_error(stream=None):
     detail = (_i32 * 3)()
     status = lib().mla_get_device_error(_stream(stream), detail)
     return status, list(detail)
+
+
+def mla_check_wait_timeout(limit_ns: int, stream=None):
+    """Launch the library's bounded-wait check (a wait that must give up after ``limit_ns``)."""
+    _check(lib().mla_check_wait_timeout(int(limit_ns), _stream(stream)), "mla_check_wait_timeout")
 
 
 def mla_kernel_launches() -> int:

@@ -10,7 +10,7 @@
 #include "common.cuh"
 #include "decode_plan.cuh"
 #include "decode_simt.cuh"
-#include "decode_tc.cuh"
+#include "decode_pair.cuh"
 #include "elementwise.cuh"
 #include "gemm_simt.cuh"
 #include "wgemm_tc.cuh"
@@ -310,8 +310,11 @@ int default_workers(const mla_config* c) {
 // The tensor-core decode reads the query as bf16 rows [H, d_c + d_r] that a
 // first kernel packs from the fp32 inputs into the workspace.
 size_t qpack_row_bytes(const mla_config* c) {
-  return c->dtype == MLA_BF16 ? (size_t)c->n_heads * (c->d_c + c->d_r) * 2 : 0;
+  return c->dtype == MLA_BF16 ? pairdec::qpack_row_bytes(c) : 0;
 }
+
+// Time limit of every bounded wait in the tensor-core decode (process-wide).
+std::atomic<unsigned long long> g_wait_limit_ns{sm100::kWaitLimitNs};
 
 int resolve_workers(const mla_config* c, int max_workers) {
   return max_workers > 0 ? max_workers : default_workers(c);
@@ -370,6 +373,21 @@ mla_status append_scratch_address(void** out) {
   }
   *out = p;
   return MLA_OK;
+}
+
+// A barrier that expects two arrivals and gets one: the bounded wait on it
+// must give up after `limit_ns`, record MLA_ERR_TIMEOUT (where = 1) and return.
+__global__ void wait_timeout_check_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 2);
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    sm100::mbar_arrive(&bar);  // the second arrival never comes
+    sm100::mbar_wait(&bar, 0, 1, limit_ns);
+  }
 }
 
 }  // namespace
@@ -475,24 +493,22 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
   if ((long long)batch * n_q > kPlanMaxRows) return MLA_ERR_UNSUPPORTED;
   MLA_TRY(check_cache(cache));
   if (cache->batch < batch) return MLA_ERR_INVALID_ARG;
-  if (cfg->dtype == MLA_BF16 && !tcdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
+  if (cfg->dtype == MLA_BF16 && !pairdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
   if (cfg->dtype == MLA_BF16 && !all_aligned16(q_lat, q_rope, cache->pool, workspace)) return MLA_ERR_INVALID_ARG;
   const DecodeLayout L =
       decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers), qpack_row_bytes(cfg));
   if (ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t plan_smem = sizeof(int) * ((size_t)batch * n_q + 1);
-  const bool fused_plan = cfg->dtype == MLA_BF16 && !(cfg->flags & MLA_FLAG_SPLIT_QUERY);
-  if (!fused_plan) {
-    if (plan_smem > 48 * 1024 &&
-        cudaFuncSetAttribute(decode_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan_smem) !=
-            cudaSuccess)
-      return MLA_ERR_CUDA;
-    MLA_CUDA(launch_chained(decode_plan_kernel, dim3(1), dim3(1024), plan_smem, s, seq_lens, cfg->block_size,
-                            cache->max_blocks_per_seq, workspace, L));
-  }
   if (cfg->dtype == MLA_BF16)
-    return tcdec::launch(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, scale_of(cfg), s, plan_smem);
+    return pairdec::launch(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, scale_of(cfg),
+                           g_wait_limit_ns.load(std::memory_order_relaxed), s);
+  const size_t plan_smem = sizeof(int) * ((size_t)batch * n_q + 1);
+  if (plan_smem > 48 * 1024 &&
+      cudaFuncSetAttribute(decode_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan_smem) !=
+          cudaSuccess)
+    return MLA_ERR_CUDA;
+  MLA_CUDA(launch_chained(decode_plan_kernel, dim3(1), dim3(1024), plan_smem, s, seq_lens, cfg->block_size,
+                          cache->max_blocks_per_seq, workspace, L));
   return decode_simt_dispatch<float>(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, s);
 }
 
@@ -531,6 +547,14 @@ mla_status mla_out_proj(const mla_config* cfg, const float* o_lat, int32_t n_tok
   }
   if (ws_bytes < out_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
   return out_impl<float>(cfg, o_lat, n_tok, W_UV, W_O, y, workspace, s);
+}
+
+mla_status mla_check_wait_timeout(int64_t limit_ns, void* stream) {
+  if (limit_ns <= 0 || limit_ns > 10000000000LL) return MLA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  wait_timeout_check_kernel<<<1, 32, 0, s>>>((unsigned long long)limit_ns);
+  note_launch();
+  return st(cudaGetLastError());
 }
 
 mla_status mla_get_device_error(void* stream, int32_t* detail) {
