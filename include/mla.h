@@ -215,6 +215,31 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
                       void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Steps 2 and 3 with the query handed over in the decode's own layout
+ * (tensor-core path, bf16 storage).  mla_absorb_q_packed computes the same
+ * absorbed query as mla_absorb_q but writes it straight from the projection's
+ * accumulators as bf16 rows, one per (token, head), of d_c + d_r values:
+ * q_lat then the rotated q_rope; in split-query mode (MLA_FLAG_SPLIT_QUERY)
+ * a second array of the same shape follows with the bf16 remainders
+ * (value - bf16(value)).  mla_decode_packed reads that buffer directly
+ * (mla_decode would first convert fp32 q_lat / q_rope into it).  The
+ * rounding is the one mla_decode applies, so results are identical.
+ *   q_packed  bf16 [n_tok, H, d_c + d_r] (x2 in split-query mode):
+ *             mla_query_packed_bytes(cfg, n_tok) bytes, 16-byte aligned
+ *   Other arguments as in mla_absorb_q / mla_decode; the decode workspace
+ *   is sized by mla_decode_workspace_size (its query region stays unused).
+ * MLA_ERR_UNSUPPORTED for fp32 storage or shapes without the tensor-core path.
+ * ------------------------------------------------------------------------- */
+size_t mla_query_packed_bytes(const mla_config* cfg, int32_t n_tok);
+mla_status mla_absorb_q_packed(const mla_config* cfg, const void* x, int32_t n_tok,
+                               const void* W_DQ, const void* W_UQ, const void* W_UK,
+                               const int32_t* pos, void* q_packed,
+                               void* workspace, size_t ws_bytes, void* stream);
+mla_status mla_decode_packed(const mla_config* cfg, const void* q_packed, int32_t batch, int32_t n_q,
+                             const mla_cache* cache, const int32_t* seq_lens, int32_t max_workers,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Step 4a - split combine (not on the pages; the standard log-sum-exp merge):
  *   o_lat[t,h] = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),  M = max_s lse_s
  * over the partials that mla_decode left in `workspace` (same batch, n_q).
@@ -238,6 +263,31 @@ size_t mla_out_proj_workspace_size(const mla_config* cfg, int32_t n_tok);
 mla_status mla_out_proj(const mla_config* cfg, const float* o_lat, int32_t n_tok,
                         const void* W_UV, const void* W_O, void* y,
                         void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Steps 4a + 4b fused - split combine inside the W_UV projection, then W_O
+ * ([P5] section 1 "Định nghĩa": W_UV folded into the output side; the merge
+ * of the splits is the standard log-sum-exp merge, not on the pages).  Since
+ * o_h = o_lat_h W_UV_h is linear in o_lat, W_UV_h is applied to every
+ * segment's partial output and the segments of a row are merged on the
+ * projection's fp32 accumulators:
+ *   o_h[t] = sum_s w_s,h (O_s,h W_UV_h),  w_s,h = 2^(lse_s,h - M) / sum_s' 2^(lse_s',h - M)
+ *   y[t]   = concat_h(o_h[t]) W_O
+ * The latent output o_lat is never written (use mla_combine for it).
+ *   decode_ws: the workspace of the mla_decode call of this step (same
+ *              batch, n_q and max_workers); read only.
+ *   W_UV [d_c, H v_head];  W_O [H v_head, hidden];  y [batch n_q, hidden] (out)
+ *   workspace >= mla_combine_out_proj_workspace_size(cfg, batch, n_q) bytes
+ * bf16 storage only (MLA_ERR_UNSUPPORTED otherwise, or when v_head != 128 or
+ * the decode has more than 512 segments: batch n_q + workers - 1 > 512).
+ * A decode workspace that mla_decode did not write for this batch makes y
+ * zero and records MLA_ERR_WORKSPACE on the device error word.
+ * ------------------------------------------------------------------------- */
+size_t mla_combine_out_proj_workspace_size(const mla_config* cfg, int32_t batch, int32_t n_q);
+mla_status mla_combine_out_proj(const mla_config* cfg, const void* decode_ws, size_t decode_ws_bytes,
+                                int32_t batch, int32_t n_q, int32_t max_workers,
+                                const void* W_UV, const void* W_O, void* y,
+                                void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Errors and introspection

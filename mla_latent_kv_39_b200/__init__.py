@@ -12,16 +12,21 @@ from .abi import (  # noqa: F401
     check_device_error,
     lib,
     mla_absorb_q,
+    mla_absorb_q_packed,
     mla_absorb_q_workspace_size,
     mla_cache_append,
     mla_cache_append_workspace_size,
     mla_cache_append_noalloc,
     mla_combine,
+    mla_combine_out_proj,
+    mla_combine_out_proj_workspace_size,
     mla_decode,
+    mla_decode_packed,
     mla_decode_workspace_size,
     mla_get_device_error,
     mla_kernel_launches,
     mla_out_proj,
     mla_out_proj_workspace_size,
+    mla_query_packed_bytes,
 )
 from .layer import DecodeLayer  # noqa: F401

@@ -63,9 +63,14 @@ SIGNATURES = {
     "mla_cache_append_noalloc": (_i32, [_P_CFG, _vp, _i32, _vp, _vp, _vp, _vp, _P_CACHE, _vp]),
     "mla_absorb_q_workspace_size": (_sz, [_P_CFG, _i32]),
     "mla_absorb_q": (_i32, [_P_CFG, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "mla_query_packed_bytes": (_sz, [_P_CFG, _i32]),
+    "mla_absorb_q_packed": (_i32, [_P_CFG, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "mla_decode_packed": (_i32, [_P_CFG, _vp, _i32, _i32, _P_CACHE, _vp, _i32, _vp, _sz, _vp]),
     "mla_decode_workspace_size": (_sz, [_P_CFG, _i32, _i32, _i32]),
     "mla_decode": (_i32, [_P_CFG, _vp, _vp, _i32, _i32, _P_CACHE, _vp, _i32, _vp, _sz, _vp]),
     "mla_combine": (_i32, [_P_CFG, _vp, _sz, _i32, _i32, _vp, _vp]),
+    "mla_combine_out_proj_workspace_size": (_sz, [_P_CFG, _i32, _i32]),
+    "mla_combine_out_proj": (_i32, [_P_CFG, _vp, _sz, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mla_out_proj_workspace_size": (_sz, [_P_CFG, _i32]),
     "mla_out_proj": (_i32, [_P_CFG, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mla_get_device_error": (_i32, [_vp, ctypes.POINTER(_i32)]),
@@ -254,6 +259,44 @@ def mla_absorb_q(cfg: Config, x, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, workspace
                               _stream(stream)), "mla_absorb_q")
 
 
+def mla_query_packed_bytes(cfg: Config, n_tok: int) -> int:
+    return int(lib().mla_query_packed_bytes(ctypes.byref(cfg.c()), n_tok))
+
+
+def mla_absorb_q_packed(cfg: Config, x, W_DQ, W_UQ, W_UK, pos, q_packed, workspace, stream=None):
+    dt = cfg.torch_dtype
+    n = x.shape[0]
+    H = cfg.n_heads
+    _need(x, "x", dt, shape=(n, cfg.hidden))
+    if cfg.q_lora > 0:
+        _need(W_DQ, "W_DQ", dt, shape=(cfg.hidden, cfg.q_lora))
+        _need(W_UQ, "W_UQ", dt, shape=(cfg.q_lora, H * (cfg.qk_nope + cfg.d_r)))
+    else:
+        if W_DQ is not None:
+            raise ValueError("W_DQ must be None without query compression")
+        _need(W_UQ, "W_Q", dt, shape=(cfg.hidden, H * (cfg.qk_nope + cfg.d_r)))
+    _need(W_UK, "W_UK", dt, shape=(cfg.d_c, H * cfg.qk_nope))
+    _need(pos, "pos", torch.int32, shape=(n,))
+    _need(q_packed, "q_packed", torch.bfloat16,
+          shape=((2 if cfg.split_query else 1) * n, H, cfg.d_c + cfg.d_r))
+    _need(workspace, "workspace", torch.uint8)
+    _check(lib().mla_absorb_q_packed(ctypes.byref(cfg.c()), _ptr(x), n, _ptr(W_DQ), _ptr(W_UQ), _ptr(W_UK),
+                                     _ptr(pos), _ptr(q_packed), _ptr(workspace), workspace.numel(),
+                                     _stream(stream)), "mla_absorb_q_packed")
+
+
+def mla_decode_packed(cfg: Config, q_packed, batch: int, n_q: int, cache: Cache, seq_lens, workspace,
+                      max_workers: int = 0, stream=None):
+    H = cfg.n_heads
+    _need(q_packed, "q_packed", torch.bfloat16,
+          shape=((2 if cfg.split_query else 1) * batch * n_q, H, cfg.d_c + cfg.d_r))
+    _need(seq_lens, "seq_lens", torch.int32, shape=(batch,))
+    _need(workspace, "workspace", torch.uint8)
+    _check(lib().mla_decode_packed(ctypes.byref(cfg.c()), _ptr(q_packed), batch, n_q, ctypes.byref(cache.c),
+                                   _ptr(seq_lens), max_workers, _ptr(workspace), workspace.numel(),
+                                   _stream(stream)), "mla_decode_packed")
+
+
 def mla_decode(cfg: Config, q_lat, q_rope, batch: int, n_q: int, cache: Cache, seq_lens, workspace,
                max_workers: int = 0, stream=None):
     dt = cfg.torch_dtype
@@ -272,6 +315,24 @@ def mla_combine(cfg: Config, workspace, batch: int, n_q: int, o_lat, stream=None
     _need(o_lat, "o_lat", torch.float32, shape=(batch * n_q, cfg.n_heads, cfg.d_c))
     _check(lib().mla_combine(ctypes.byref(cfg.c()), _ptr(workspace), workspace.numel(), batch, n_q,
                              _ptr(o_lat), _stream(stream)), "mla_combine")
+
+
+def mla_combine_out_proj_workspace_size(cfg: Config, batch: int, n_q: int) -> int:
+    return int(lib().mla_combine_out_proj_workspace_size(ctypes.byref(cfg.c()), batch, n_q))
+
+
+def mla_combine_out_proj(cfg: Config, decode_ws, batch: int, n_q: int, W_UV, W_O, y, workspace,
+                         max_workers: int = 0, stream=None):
+    dt = cfg.torch_dtype
+    H = cfg.n_heads
+    _need(decode_ws, "decode_ws", torch.uint8)
+    _need(W_UV, "W_UV", dt, shape=(cfg.d_c, H * cfg.v_head))
+    _need(W_O, "W_O", dt, shape=(H * cfg.v_head, cfg.hidden))
+    _need(y, "y", dt, shape=(batch * n_q, cfg.hidden))
+    _need(workspace, "workspace", torch.uint8)
+    _check(lib().mla_combine_out_proj(ctypes.byref(cfg.c()), _ptr(decode_ws), decode_ws.numel(), batch, n_q,
+                                      max_workers, _ptr(W_UV), _ptr(W_O), _ptr(y), _ptr(workspace),
+                                      workspace.numel(), _stream(stream)), "mla_combine_out_proj")
 
 
 def mla_out_proj(cfg: Config, o_lat, W_UV, W_O, y, workspace, stream=None):

@@ -8,14 +8,12 @@
 // fixed charge per row for the segment's setup); where a range crosses a row
 // boundary it is cut again, so every piece - a "segment" - covers pages
 // [blk_begin, blk_end) of one query row.  There are
-// at most workers + rows - 1 segments.  Each segment's decode writes, per
-// head, its output normalised over its own rows plus the log2-sum-exp of its
-// scaled scores; the combine merges the segments of a row.  The partial
-// outputs are stored head-minor ([segment][d][h]): the tensor-core decode
-// holds one head per TMEM lane, so a warp's 32 heads of one column form one
-// 128-byte store.  The plan is
-// computed on the device from seq_lens, so a decode step never waits on the
-// host.
+// at most workers + rows - 1 segments, and they are ordered by query row.
+// Each segment's decode writes, per head, its output normalised over its own
+// rows ([segment][h][d], bf16 from the tensor-core decode, fp32 from the
+// CUDA-core one) plus the log2-sum-exp of its scaled scores; the combine
+// merges the segments of a row.  The plan is computed on the device from
+// seq_lens, so a decode step never waits on the host.
 #pragma once
 
 #include "common.cuh"
@@ -26,13 +24,14 @@ constexpr int kPlanMagic = 0x4D4C4131;  // "MLA1"
 
 struct DecodeLayout {
   int batch, n_q, H, d_c, workers, max_segments;
+  int part_elem;               // bytes per partial-output value: 2 (bf16) or 4 (fp32)
   long long off_prefix;        // int32 [rows + 1]    pages before query row v
   long long off_worker_first;  // int32 [workers + 1] first segment of worker w
   long long off_seq_first;     // int32 [rows]        first segment of query row v
   long long off_seq_nseg;      // int32 [rows]        number of segments of query row v
   long long off_seg;           // int4  [max_segments] (v, blk_begin, blk_end, worker)
   long long off_lse;           // f32   [max_segments, H]        log2-sum-exp
-  long long off_o;             // f32   [max_segments, d_c, H]   normalised partial output (head-minor)
+  long long off_o;             // bf16 / f32 [max_segments, H, d_c]  normalised partial output
   long long off_qpack;         // bf16  [rows, H, d_c + d_r]     the query in bf16 (tensor-core path)
   long long total;
 };
@@ -44,9 +43,10 @@ struct DecodeHeader {
 };
 
 static inline DecodeLayout decode_layout(int batch, int n_q, int H, int d_c, int workers,
-                                         size_t qpack_row_bytes = 0) {
+                                         size_t qpack_row_bytes, int part_elem) {
   DecodeLayout L{};
   const size_t rows = (size_t)batch * n_q;
+  L.part_elem = part_elem;
   L.batch = batch;
   L.n_q = n_q;
   L.H = H;
@@ -60,7 +60,7 @@ static inline DecodeLayout decode_layout(int batch, int n_q, int H, int d_c, int
   L.off_seq_nseg = o;      o = align_up(o + sizeof(int) * rows, 256);
   L.off_seg = o;           o = align_up(o + sizeof(int4) * (size_t)L.max_segments, 256);
   L.off_lse = o;           o = align_up(o + sizeof(float) * (size_t)L.max_segments * H, 256);
-  L.off_o = o;             o = align_up(o + sizeof(float) * (size_t)L.max_segments * H * d_c, 256);
+  L.off_o = o;             o = align_up(o + (size_t)part_elem * L.max_segments * H * d_c, 256);
   L.off_qpack = o;         o = align_up(o + qpack_row_bytes * rows, 256);
   L.total = o;
   return L;
@@ -226,59 +226,77 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
   plan_body(seq_lens, bs, max_blocks, ws, L);
 }
 
-// o_lat[v, h, d] = sum_s 2^(lse_s,h - M_h) O_s[d, h] / sum_s 2^(lse_s,h - M_h)
-// over the segments s of query row v (M_h the largest lse_s,h).  Grid (query
-// rows, d_c / 32 column blocks), one thread per head (looping past 128 heads);
-// the 32-column x 128-head tile goes through shared memory, so the partial
-// outputs are read head-minor and o_lat is written column-minor, both in
-// whole 128-byte lines.
-constexpr int kCombDims = 32;
-__global__ void __launch_bounds__(128) combine_kernel(const void* ws, long long ws_bytes, int batch,
-                                                      int n_q, int H, int d_c, float* __restrict__ o_lat) {
+// Weight of segment `first + s` in the merge of query row v for head h:
+// 2^(lse_s - M) / sum_s' 2^(lse_s' - M) with M the largest lse of the row.
+struct RowMerge {
+  float M, invZ;
+  __device__ RowMerge(const float* lse, int first, int n, int H, int h) : M(-INFINITY), invZ(0.f) {
+    for (int s = 0; s < n; ++s) M = fmaxf(M, lse[(long long)(first + s) * H + h]);
+    if (M == -INFINITY) return;
+    float Z = 0.f;
+    for (int s = 0; s < n; ++s) Z += exp2f(lse[(long long)(first + s) * H + h] - M);
+    invZ = 1.f / Z;
+  }
+  __device__ float weight(float lse_s) const { return invZ > 0.f ? exp2f(lse_s - M) * invZ : 0.f; }
+};
+
+__device__ __forceinline__ void load8(const float* p, float (&x)[8]) {
+  const float4 a = __ldcs(reinterpret_cast<const float4*>(p)), b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ void load8(const bf16* p, float (&x)[8]) {
+  const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    x[2 * k] = __uint_as_float(w[k] << 16);
+    x[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+  }
+}
+
+// o_lat[v, h, d] = sum_s w_s,h O_s[h, d] over the segments s of query row v.
+// Grid (query rows, head blocks); a thread owns 8 consecutive d of one head
+// (d_c / 8 threads per head), so every load and store is a 16- or 32-byte
+// vector and a warp covers whole rows.
+// With `valid` false (a workspace no decode wrote) the row is written as zeros.
+template <typename P>
+__device__ void combine_rows(const void* ws, const DecodeLayout& L, bool valid, int v, int H, int d_c,
+                             float* __restrict__ o_lat) {
+  const int per_head = d_c / 8;
+  const int hb = blockDim.x / per_head;
+  const int h = blockIdx.y * hb + threadIdx.x / per_head, d0 = 8 * (threadIdx.x % per_head);
+  if (h >= H || threadIdx.x >= hb * per_head) return;
+  const int first = valid ? ws_at<int>(ws, L.off_seq_first)[v] : 0;
+  const int n = valid ? ws_at<int>(ws, L.off_seq_nseg)[v] : 0;
+  const float* lse = ws_at<float>(ws, L.off_lse);
+  const P* part = ws_at<P>(ws, L.off_o);
+  const RowMerge rm(lse, first, n, H, h);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < n; ++s) {
+    const float w = rm.weight(lse[(long long)(first + s) * H + h]);
+    if (w == 0.f) continue;  // no rows in this piece: its output was never written
+    float x[8];
+    load8(part + ((long long)(first + s) * H + h) * d_c + d0, x);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = fmaf(w, x[k], acc[k]);
+  }
+  float* out = o_lat + ((long long)v * H + h) * d_c + d0;
+  *reinterpret_cast<float4*>(out) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  *reinterpret_cast<float4*>(out + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+__global__ void __launch_bounds__(256) combine_kernel(const void* ws, long long ws_bytes, int batch, int n_q, int H,
+                                                      int d_c, float* __restrict__ o_lat) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float tile[kCombDims][129];
   const DecodeHeader* hd = ws_at<DecodeHeader>(ws, 0);
-  const int v = blockIdx.x, d0 = blockIdx.y * kCombDims, nd = min(kCombDims, d_c - d0);
   const bool bad = hd->magic != kPlanMagic || hd->batch != batch || hd->n_q != n_q || hd->H != H ||
                    hd->d_c != d_c || hd->layout.total > ws_bytes;
+  const int v = blockIdx.x;
   if (bad && v == 0 && blockIdx.y == 0 && threadIdx.x == 0) report(MLA_ERR_WORKSPACE, 0, batch, n_q);
   const DecodeLayout L = hd->layout;
-  const int first = bad ? 0 : ws_at<int>(ws, L.off_seq_first)[v];
-  const int n = bad ? 0 : ws_at<int>(ws, L.off_seq_nseg)[v];
-  const float* lse = ws_at<float>(ws, L.off_lse);
-  const float* part = ws_at<float>(ws, L.off_o);
-  for (int h0 = 0; h0 < H; h0 += 128) {
-    const int h = h0 + threadIdx.x;
-    float acc[kCombDims];
-#pragma unroll
-    for (int i = 0; i < kCombDims; ++i) acc[i] = 0.f;
-    if (h < H && n > 0) {
-      float M = -INFINITY;
-      for (int s = 0; s < n; ++s) M = fmaxf(M, lse[(long long)(first + s) * H + h]);
-      if (M != -INFINITY) {
-        float Z = 0.f;
-        for (int s = 0; s < n; ++s) Z += exp2f(lse[(long long)(first + s) * H + h] - M);
-        const float invZ = 1.f / Z;
-        for (int s = 0; s < n; ++s) {
-          const long long seg = first + s;
-          const float w = exp2f(lse[seg * H + h] - M) * invZ;
-          const float* src = part + (seg * d_c + d0) * H + h;
-#pragma unroll
-          for (int i = 0; i < kCombDims; ++i)
-            if (i < nd) acc[i] = fmaf(w, __ldcs(src + (long long)i * H), acc[i]);
-        }
-      }
-    }
-    __syncthreads();  // the previous head block's tile has been written out
-#pragma unroll
-    for (int i = 0; i < kCombDims; ++i) tile[i][threadIdx.x] = acc[i];
-    __syncthreads();
-    for (int e = threadIdx.x; e < 128 * kCombDims; e += 128) {
-      const int hh = e / kCombDims, i = e % kCombDims;
-      if (h0 + hh < H && i < nd) o_lat[((long long)v * H + h0 + hh) * d_c + d0 + i] = tile[i][hh];
-    }
-  }
+  if (!bad && L.part_elem == 2) combine_rows<bf16>(ws, L, true, v, H, d_c, o_lat);
+  else combine_rows<float>(ws, L, !bad, v, H, d_c, o_lat);
 }
 
 }  // namespace mla

@@ -74,11 +74,11 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(
   }
   const long long r_out = (long long)sidx * H + h;
   const float inv = l > 0.f ? 1.f / l : 0.f;
-  float* out = ws_at<float>(ws, L.off_o) + (long long)sidx * d_c * H + h;  // head-minor
+  float* out = ws_at<float>(ws, L.off_o) + r_out * d_c;  // [segment][h][d]
 #pragma unroll
   for (int i = 0; i < DPL; ++i) {
     const int d = lane + 32 * i;
-    if (d < d_c) out[(long long)d * H] = o[i] * inv;
+    if (d < d_c) out[d] = o[i] * inv;
   }
   if (lane == 0) ws_at<float>(ws, L.off_lse)[r_out] = l > 0.f ? m + log2f(l) : -INFINITY;
 }

@@ -117,14 +117,18 @@ __global__ void query_split_kernel(const float* __restrict__ q, int n_tok, int H
 }
 
 // Split q [n, H, nope + d_r] (fp32): q_nope to bf16 (and its bf16 remainder
-// when lo != nullptr), the rotated q_rope kept in fp32 (angle and rotation in
-// fp64).  One block per (token, group of kHeadGroup heads): the token's d_r/2
-// rotation angles are evaluated once into shared memory and shared by every
-// head.  Needs even nope and d_r (pairs are read and written together).
+// when lo != nullptr), the rotated q_rope (angle and rotation in fp64) kept
+// in fp32 (q_rope) and/or written as bf16 (and its remainder) into columns
+// [rope_col, rope_col + d_r) of the packed query rows of `row` values
+// (qp_hi / qp_lo).  One block per (token, group of kHeadGroup heads): the
+// token's d_r/2 rotation angles are evaluated once into shared memory and
+// shared by every head.  Needs even nope and d_r (pairs are read and written
+// together).
 constexpr int kHeadGroup = 8;
 __global__ void query_split_bf16_kernel(const float* __restrict__ q, int n_tok, int H, int nope, int d_r,
                                         double theta, const int32_t* __restrict__ pos, bf16* __restrict__ q_nope,
-                                        bf16* __restrict__ q_nope_lo, float* __restrict__ q_rope) {
+                                        bf16* __restrict__ q_nope_lo, float* __restrict__ q_rope,
+                                        bf16* __restrict__ qp_hi, bf16* __restrict__ qp_lo, int row, int rope_col) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ double rot[];  // [d_r/2][cos, sin]
@@ -153,8 +157,17 @@ __global__ void query_split_bf16_kernel(const float* __restrict__ q, int n_tok, 
     const int pr = e % half;
     const float2 r = *reinterpret_cast<const float2*>(q + th * w + nope + 2 * pr);
     const double cs = rot[2 * pr], sn = rot[2 * pr + 1];
-    *reinterpret_cast<float2*>(q_rope + th * d_r + 2 * pr) =
+    const float2 rr =
         make_float2((float)((double)r.x * cs - (double)r.y * sn), (float)((double)r.x * sn + (double)r.y * cs));
+    if (q_rope) *reinterpret_cast<float2*>(q_rope + th * d_r + 2 * pr) = rr;
+    if (qp_hi) {
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(rr.x, rr.y);
+      const long long o = th * row + rope_col + 2 * pr;
+      *reinterpret_cast<__nv_bfloat162*>(qp_hi + o) = hi;
+      if (qp_lo)
+        *reinterpret_cast<__nv_bfloat162*>(qp_lo + o) =
+            __floats2bfloat162_rn(rr.x - __bfloat162float(hi.x), rr.y - __bfloat162float(hi.y));
+    }
   }
 }
 

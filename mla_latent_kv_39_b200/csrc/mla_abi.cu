@@ -13,6 +13,7 @@
 #include "decode_pair.cuh"
 #include "elementwise.cuh"
 #include "gemm_simt.cuh"
+#include "out_combine.cuh"
 #include "wgemm_tc.cuh"
 
 using namespace mla;
@@ -244,8 +245,13 @@ AbsorbTcWs absorb_tc_ws(const mla_config* c, int n) {
   return w;
 }
 
+// Query side on the tensor cores.  Outputs either fp32 q_lat / q_rope, or
+// (q_packed != nullptr) the decode's packed bf16 rows [n][H][d_c + d_r]
+// (q_lat then the rotated q_R), followed in split-query mode by a second
+// such array with the bf16 remainders.
 mla_status absorb_tc(const mla_config* c, const void* x, int n, const void* W_DQ, const void* W_UQ,
-                     const void* W_UK, const int32_t* pos, float* q_lat, float* q_rope, void* ws, cudaStream_t s) {
+                     const void* W_UK, const int32_t* pos, float* q_lat, float* q_rope, bf16* q_packed, void* ws,
+                     cudaStream_t s) {
   const bool split = (c->flags & MLA_FLAG_SPLIT_QUERY) != 0;
   const AbsorbTcWs w = absorb_tc_ws(c, n);
   char* base = static_cast<char*>(ws);
@@ -259,11 +265,16 @@ mla_status absorb_tc(const mla_config* c, const void* x, int n, const void* W_DQ
                                   cq_hi, cq_lo, qn_hi, qn_lo, nullptr, nullptr);
   if (c->q_lora > 0) MLA_TRY(wg::run(ps.dq, part, nullptr, cq_hi, cq_lo, s));
   MLA_TRY(wg::run(ps.uq, part, q_f, nullptr, nullptr, s));
-  const int H = c->n_heads, nope = c->qk_nope;
+  const int H = c->n_heads, nope = c->qk_nope, row = c->d_c + c->d_r;
+  bf16* qp_lo = q_packed && split ? q_packed + (long long)n * H * row : nullptr;
   const dim3 qgrid(n, (H + kHeadGroup - 1) / kHeadGroup);
   MLA_CUDA(launch_chained(query_split_bf16_kernel, qgrid, dim3(256), sizeof(double) * c->d_r, s, (const float*)q_f, n, H,
-                          nope, c->d_r, c->rope_theta, pos, qn_hi, qn_lo, q_rope));
-  return wg::run(ps.uk, part, q_lat, nullptr, nullptr, s);
+                          nope, c->d_r, c->rope_theta, pos, qn_hi, qn_lo, q_rope, q_packed, qp_lo, row, c->d_c));
+  if (q_packed == nullptr) return wg::run(ps.uk, part, q_lat, nullptr, nullptr, s);
+  wg::Spec uk = ps.uk;  // q_lat of head h of token t -> packed row t H + h, columns [0, d_c)
+  uk.o_ts = (long long)H * row;
+  uk.o_gs = row;
+  return wg::run(uk, part, nullptr, q_packed, qp_lo, s);
 }
 
 struct OutTcWs {
@@ -312,6 +323,10 @@ int default_workers(const mla_config* c) {
 size_t qpack_row_bytes(const mla_config* c) {
   return c->dtype == MLA_BF16 ? pairdec::qpack_row_bytes(c) : 0;
 }
+
+// Partial outputs of the split decode: bf16 from the tensor-core decode
+// (they feed bf16 MMAs next), fp32 from the CUDA-core one.
+int part_elem(const mla_config* c) { return c->dtype == MLA_BF16 ? 2 : 4; }
 
 // Time limit of every bounded wait in the tensor-core decode (process-wide).
 std::atomic<unsigned long long> g_wait_limit_ns{sm100::kWaitLimitNs};
@@ -470,16 +485,56 @@ mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok, con
     if (!proj_tc_supported(cfg)) return MLA_ERR_UNSUPPORTED;
     if (!all_aligned16(x, W_DQ, W_UQ, W_UK, q_lat, q_rope, workspace)) return MLA_ERR_INVALID_ARG;
     if (ws_bytes < absorb_tc_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
-    return absorb_tc(cfg, x, n_tok, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, workspace, s);
+    return absorb_tc(cfg, x, n_tok, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, nullptr, workspace, s);
   }
   if (ws_bytes < absorb_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
   return absorb_impl<float>(cfg, x, n_tok, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, workspace, s);
 }
 
+size_t mla_query_packed_bytes(const mla_config* cfg, int32_t n_tok) {
+  if (check_cfg(cfg) != MLA_OK || n_tok < 0 || cfg->dtype != MLA_BF16) return 0;
+  return (size_t)n_tok * pairdec::qpack_row_bytes(cfg);
+}
+
+mla_status mla_absorb_q_packed(const mla_config* cfg, const void* x, int32_t n_tok, const void* W_DQ,
+                               const void* W_UQ, const void* W_UK, const int32_t* pos, void* q_packed,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  MLA_TRY(check_cfg(cfg));
+  if (n_tok < 0) return MLA_ERR_INVALID_ARG;
+  if (n_tok == 0) return MLA_OK;
+  if (!x || !W_UQ || !W_UK || !pos || !q_packed || !workspace) return MLA_ERR_INVALID_ARG;
+  if ((cfg->q_lora > 0) != (W_DQ != nullptr)) return MLA_ERR_INVALID_ARG;
+  if (cfg->dtype != MLA_BF16 || !proj_tc_supported(cfg) || !pairdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
+  if (!all_aligned16(x, W_DQ, W_UQ, W_UK, q_packed, workspace)) return MLA_ERR_INVALID_ARG;
+  if (ws_bytes < absorb_tc_ws(cfg, n_tok).total) return MLA_ERR_WORKSPACE;
+  return absorb_tc(cfg, x, n_tok, W_DQ, W_UQ, W_UK, pos, nullptr, nullptr, static_cast<bf16*>(q_packed), workspace,
+                   static_cast<cudaStream_t>(stream));
+}
+
+mla_status mla_decode_packed(const mla_config* cfg, const void* q_packed, int32_t batch, int32_t n_q,
+                             const mla_cache* cache, const int32_t* seq_lens, int32_t max_workers, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  MLA_TRY(check_cfg(cfg));
+  if (batch < 0 || n_q <= 0 || max_workers < 0) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!q_packed || !seq_lens || !workspace) return MLA_ERR_INVALID_ARG;
+  if ((long long)batch * n_q > kPlanMaxRows) return MLA_ERR_UNSUPPORTED;
+  MLA_TRY(check_cache(cache));
+  if (cache->batch < batch) return MLA_ERR_INVALID_ARG;
+  if (cfg->dtype != MLA_BF16 || !pairdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
+  if (!all_aligned16(q_packed, cache->pool, workspace)) return MLA_ERR_INVALID_ARG;
+  const DecodeLayout L = decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers),
+                                       qpack_row_bytes(cfg), part_elem(cfg));
+  if (ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
+  return pairdec::launch(cfg, nullptr, nullptr, static_cast<const bf16*>(q_packed), n_q, cache, seq_lens, workspace,
+                         L, scale_of(cfg), g_wait_limit_ns.load(std::memory_order_relaxed),
+                         static_cast<cudaStream_t>(stream));
+}
+
 size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t n_q, int32_t max_workers) {
   if (check_cfg(cfg) != MLA_OK || batch < 0 || n_q <= 0 || max_workers < 0) return 0;
   return (size_t)decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers),
-                               qpack_row_bytes(cfg))
+                               qpack_row_bytes(cfg), part_elem(cfg))
       .total;
 }
 
@@ -496,11 +551,12 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
   if (cfg->dtype == MLA_BF16 && !pairdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
   if (cfg->dtype == MLA_BF16 && !all_aligned16(q_lat, q_rope, cache->pool, workspace)) return MLA_ERR_INVALID_ARG;
   const DecodeLayout L =
-      decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers), qpack_row_bytes(cfg));
+      decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers), qpack_row_bytes(cfg),
+                    part_elem(cfg));
   if (ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cfg->dtype == MLA_BF16)
-    return pairdec::launch(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, scale_of(cfg),
+    return pairdec::launch(cfg, q_lat, q_rope, nullptr, n_q, cache, seq_lens, workspace, L, scale_of(cfg),
                            g_wait_limit_ns.load(std::memory_order_relaxed), s);
   const size_t plan_smem = sizeof(int) * ((size_t)batch * n_q + 1);
   if (plan_smem > 48 * 1024 &&
@@ -519,11 +575,48 @@ mla_status mla_combine(const mla_config* cfg, const void* workspace, size_t ws_b
   if (batch == 0) return MLA_OK;
   if (!workspace || !o_lat) return MLA_ERR_INVALID_ARG;
   if (ws_bytes < sizeof(DecodeHeader)) return MLA_ERR_WORKSPACE;
-  if (cfg->dtype == MLA_BF16 && !all_aligned16(workspace, o_lat)) return MLA_ERR_INVALID_ARG;
+  if (!all_aligned16(workspace, o_lat)) return MLA_ERR_INVALID_ARG;
+  if (cfg->d_c % 8 != 0 || cfg->d_c / 8 > 256) return MLA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  dim3 grid(batch * n_q, (cfg->d_c + kCombDims - 1) / kCombDims);
-  return st(launch_chained(combine_kernel, grid, dim3(128), 0, s, (const void*)workspace, (long long)ws_bytes, batch,
+  const int per_head = cfg->d_c / 8, heads_per_block = 256 / per_head;
+  dim3 grid(batch * n_q, (cfg->n_heads + heads_per_block - 1) / heads_per_block);
+  return st(launch_chained(combine_kernel, grid, dim3(256), 0, s, (const void*)workspace, (long long)ws_bytes, batch,
                             n_q, cfg->n_heads, cfg->d_c, o_lat));
+}
+
+size_t mla_combine_out_proj_workspace_size(const mla_config* cfg, int32_t batch, int32_t n_q) {
+  if (check_cfg(cfg) != MLA_OK || batch < 0 || n_q <= 0 || cfg->dtype != MLA_BF16 || !proj_tc_supported(cfg))
+    return 0;
+  const int n = batch * n_q;
+  const ProjSpecs ps = proj_specs(cfg, n, false, nullptr, nullptr, nullptr, nullptr, nullptr, kSizeOnly, kSizeOnly,
+                                  kSizeOnly, kSizeOnly, kSizeOnly, kSizeOnly, kSizeOnly);
+  return align_up(2 * (size_t)n * cfg->n_heads * cfg->v_head, 256) + align_up(wg::run_partial_bytes(ps.o), 256);
+}
+
+mla_status mla_combine_out_proj(const mla_config* cfg, const void* decode_ws, size_t decode_ws_bytes, int32_t batch,
+                                int32_t n_q, int32_t max_workers, const void* W_UV, const void* W_O, void* y,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  MLA_TRY(check_cfg(cfg));
+  if (batch < 0 || n_q <= 0 || max_workers < 0) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!decode_ws || !W_UV || !W_O || !y || !workspace) return MLA_ERR_INVALID_ARG;
+  if (cfg->dtype != MLA_BF16 || !proj_tc_supported(cfg) || !pairdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
+  if (!all_aligned16(decode_ws, W_UV, W_O, y, workspace)) return MLA_ERR_INVALID_ARG;
+  if ((long long)batch * n_q > kPlanMaxRows) return MLA_ERR_UNSUPPORTED;
+  const DecodeLayout L = decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers),
+                                       qpack_row_bytes(cfg), part_elem(cfg));
+  if (decode_ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
+  if (!ocomb::supports(cfg, L.max_segments)) return MLA_ERR_UNSUPPORTED;
+  if (ws_bytes < mla_combine_out_proj_workspace_size(cfg, batch, n_q)) return MLA_ERR_WORKSPACE;
+  const int n = batch * n_q;
+  char* base = static_cast<char*>(workspace);
+  bf16* oh = reinterpret_cast<bf16*>(base);
+  float* part = reinterpret_cast<float*>(base + align_up(2 * (size_t)n * cfg->n_heads * cfg->v_head, 256));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MLA_TRY(ocomb::launch(cfg, W_UV, decode_ws, decode_ws_bytes, L, oh, s));
+  const ProjSpecs ps = proj_specs(cfg, n, false, nullptr, nullptr, nullptr, W_UV, W_O, nullptr, nullptr, nullptr,
+                                  nullptr, nullptr, nullptr, oh);
+  return wg::run(ps.o, part, nullptr, static_cast<bf16*>(y), nullptr, s);
 }
 
 size_t mla_out_proj_workspace_size(const mla_config* cfg, int32_t n_tok) {

@@ -49,6 +49,15 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// Arrive on the barrier at `cluster_addr` (a shared::cluster address, e.g. in
+// the leader CTA of a pair) with the default (CTA-scope) semantics; cheap,
+// unlike a release at cluster scope.  Generic-proxy shared-memory writes
+// meant for the tensor cores are ordered by fence.proxy.async before it, and
+// TMEM accesses by tcgen05.fence::before_thread_sync.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -90,13 +99,36 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // Wait for phase `parity` of `bar` to complete; false after `limit_ns` (the
 // caller then aborts its role and the kernel returns MLA_ERR_TIMEOUT).
+__device__ __forceinline__ bool mbar_test_acq_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Build-time choice of the polling instruction: try_wait (the thread may be
+// suspended until the phase completes) or test_wait (pure polling).
+#ifndef MLA_WAIT_POLL
+#define MLA_WAIT_POLL 0
+#endif
+template <bool kCluster>
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) {
+  if (MLA_WAIT_POLL) return kCluster ? mbar_test_acq_cluster(bar, parity) : mbar_test(bar, parity);
+  return kCluster ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity);
+}
+
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int where,
                                           uint64_t limit_ns = kWaitLimitNs) {
-  if (kCluster ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  if (mbar_poll<kCluster>(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 0;; ++it) {
-    if (kCluster ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if (mbar_poll<kCluster>(bar, parity)) return true;
     if ((it & 255u) == 255u && global_ns() - t0 > limit_ns) {
       report(MLA_ERR_TIMEOUT, where, (int)blockIdx.x, (int)threadIdx.x);
       return false;
@@ -117,6 +149,12 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
       ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// Pull a tile of a 3-D tensor map into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void prefetch_l2_3d(const CUtensorMap* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y), "r"(z)
+               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
@@ -267,6 +305,18 @@ __device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, ui
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] x B[smem desc] over the CTA pair: each CTA's rows of
+// A sit in its TMEM lanes 0..63 and again in lanes 64..127.
+__device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 

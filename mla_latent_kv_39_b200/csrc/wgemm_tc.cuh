@@ -63,9 +63,10 @@ struct Params {
   int split;            // B has a lo part
   int F;                // features per group
   float* part;          // [S][n_tok][G][F] (S > 1)
-  float* out_f32;       // with S == 1 the accumulator goes straight to the outputs [n_tok][G][F]
+  float* out_f32;       // with S == 1 the accumulator goes straight to the outputs
   bf16* out_hi;
   bf16* out_lo;
+  long long o_ts, o_gs;  // output element (t, g, f) at t o_ts + g o_gs + f
 };
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
@@ -244,6 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const long long tstride = (long long)p.G * p.F;
       const long long col = (long long)g * p.F + mt * 128 + f_local;
+      const long long ocol = (long long)g * p.o_gs + mt * 128 + f_local;
       float* out = p.part + (long long)s * p.n_tok * tstride + col;
       for (int c = 0; c < p.N; c += 32) {
         uint32_t v[32];
@@ -258,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < 32; ++t) {
             if (c + t >= p.n_tok) continue;
             const float x = __uint_as_float(v[t]);
-            const long long o = (long long)(c + t) * tstride + col;
+            const long long o = (long long)(c + t) * p.o_ts + ocol;
             if (p.out_f32) p.out_f32[o] = x;
             if (p.out_hi) {
               const bf16 h = __float2bfloat16_rn(x);
@@ -297,12 +299,13 @@ __device__ __forceinline__ void emit4(float4 v, long long i, float* out_f32, bf1
   }
 }
 
-// out[i] = sum_s part[s][i] over `count` elements (a multiple of 4), summed in
-// split order, written as fp32 and/or bf16 (hi) and/or the bf16 remainder
-// (lo = value - hi).  Four elements per thread; the S loads of a group are
-// issued before the adds so they are in flight together.
-__global__ void reduce_splits_kernel(const float* __restrict__ part, int S, long long count, float* out_f32,
-                                     bf16* out_hi, bf16* out_lo) {
+// out[t, g, f] = sum_s part[s][t][g][f] over `count` = n G F elements (F a
+// multiple of 4), summed in split order, written as fp32 and/or bf16 (hi)
+// and/or the bf16 remainder (lo = value - hi) at t o_ts + g o_gs + f.  Four
+// elements per thread; the S loads of a group are issued before the adds so
+// they are in flight together.
+__global__ void reduce_splits_kernel(const float* __restrict__ part, int S, long long count, int G, int F,
+                                     long long o_ts, long long o_gs, float* out_f32, bf16* out_hi, bf16* out_lo) {
   pdl_wait();
   pdl_trigger();
   constexpr int kBatch = 8;
@@ -323,7 +326,9 @@ __global__ void reduce_splits_kernel(const float* __restrict__ part, int S, long
           acc.w += v[b].w;
         }
     }
-    emit4(acc, i, out_f32, out_hi, out_lo);
+    const long long gf = (long long)G * F;
+    const long long o = (i / gf) * o_ts + ((i / F) % G) * o_gs + i % F;
+    emit4(acc, o, out_f32, out_hi, out_lo);
   }
 }
 
@@ -374,7 +379,11 @@ struct Spec {
   const bf16* B_lo;          // optional bf16 remainder of fp32 activations
   long long b_t_stride, b_g_stride;
   int n_tok;                 // tokens of this call (<= 256)
+  long long o_ts = 0, o_gs = 0;  // output strides (0: dense [n_tok][G][F])
 };
+
+inline long long out_ts(const Spec& s) { return s.o_ts ? s.o_ts : (long long)s.G * s.F; }
+inline long long out_gs(const Spec& s) { return s.o_gs ? s.o_gs : s.F; }
 
 inline bool spec_ok(const Spec& s) {
   return s.F % 128 == 0 && s.Kg % 64 == 0 && s.n_tok > 0 && s.G > 0;
@@ -473,7 +482,7 @@ inline mla_status run(const Spec& s0, float* part, float* out_f32, bf16* out_hi,
       c.n_tok = std::min(chunk, s0.n_tok - t0);
       c.B_hi = s0.B_hi + (long long)t0 * s0.b_t_stride;
       c.B_lo = s0.B_lo ? s0.B_lo + (long long)t0 * s0.b_t_stride : nullptr;
-      const long long o = (long long)t0 * s0.G * s0.F;
+      const long long o = (long long)t0 * out_ts(s0);
       const mla_status ms = run(c, part, out_f32 ? out_f32 + o : nullptr, out_hi ? out_hi + o : nullptr,
                                 out_lo ? out_lo + o : nullptr, st);
       if (ms != MLA_OK) return ms;
@@ -491,7 +500,7 @@ inline mla_status run(const Spec& s0, float* part, float* out_f32, bf16* out_hi,
   if (ms != MLA_OK) return ms;
   if ((ms = set_attr()) != MLA_OK) return ms;
   Params p{s.G, s.F / 128, s.Kg / 64, S, s.n_tok, N, s.a_kmajor, s.a_g_stride, s.B_lo ? 1 : 0, s.F, part,
-           out_f32, out_hi, out_lo};
+           out_f32, out_hi, out_lo, out_ts(s), out_gs(s)};
   const int items = s.G * (s.F / 128) * S;
   if (launch_chained(wgemm_kernel, dim3(std::min(items, sms)), dim3(kThreads), kSmemBytes, st, a, bh, bl, p) !=
       cudaSuccess)
@@ -499,8 +508,8 @@ inline mla_status run(const Spec& s0, float* part, float* out_f32, bf16* out_hi,
   if (S == 1) return MLA_OK;
   const long long count = (long long)s.n_tok * s.G * s.F;
   const int blocks = (int)std::min<long long>((count / 4 + 255) / 256, 8 * sms);
-  return launch_chained(reduce_splits_kernel, dim3(blocks), dim3(256), 0, st, (const float*)part, S, count, out_f32,
-                        out_hi, out_lo) == cudaSuccess
+  return launch_chained(reduce_splits_kernel, dim3(blocks), dim3(256), 0, st, (const float*)part, S, count, s.G, s.F,
+                        out_ts(s), out_gs(s), out_f32, out_hi, out_lo) == cudaSuccess
              ? MLA_OK
              : MLA_ERR_CUDA;
 }

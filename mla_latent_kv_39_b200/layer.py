@@ -18,19 +18,29 @@ from . import abi
 
 class DecodeLayer:
     def __init__(self, cfg: abi.Config, weights: Dict[str, torch.Tensor], cache: abi.Cache,
-                 batch: int, n_q: int, max_workers: int = 0):
+                 batch: int, n_q: int, max_workers: int = 0, packed_query: bool = True):
         self.cfg, self.W, self.cache = cfg, weights, cache
         self.batch, self.n_q, self.max_workers = batch, n_q, max_workers
         n = batch * n_q
         dev = cache.pool.device
         dt = cfg.torch_dtype
         H = cfg.n_heads
-        self.q_lat = torch.empty(n, H, cfg.d_c, dtype=torch.float32, device=dev)
-        self.q_rope = torch.empty(n, H, cfg.d_r, dtype=torch.float32, device=dev)
+        # bf16: the absorbed query goes from the projection to the decode in the
+        # decode's packed bf16 layout (no fp32 round trip); fp32: q_lat / q_rope
+        self.packed = packed_query and abi.mla_query_packed_bytes(cfg, n) > 0
+        if self.packed:
+            rows = (2 if cfg.split_query else 1) * n
+            self.q_packed = torch.empty(rows, H, cfg.d_c + cfg.d_r, dtype=torch.bfloat16, device=dev)
+        else:
+            self.q_lat = torch.empty(n, H, cfg.d_c, dtype=torch.float32, device=dev)
+            self.q_rope = torch.empty(n, H, cfg.d_r, dtype=torch.float32, device=dev)
         self.o_lat = torch.empty(n, H, cfg.d_c, dtype=torch.float32, device=dev)
         self.y = torch.empty(n, cfg.hidden, dtype=dt, device=dev)
+        # bf16: the split combine runs inside the W_UV projection (mla_combine_out_proj)
+        self.fused_out = cfg.dtype == "bf16" and abi.mla_combine_out_proj_workspace_size(cfg, batch, n_q) > 0
         gemm_ws = max(abi.mla_cache_append_workspace_size(cfg, n), abi.mla_absorb_q_workspace_size(cfg, n),
-                      abi.mla_out_proj_workspace_size(cfg, n))
+                      abi.mla_out_proj_workspace_size(cfg, n),
+                      abi.mla_combine_out_proj_workspace_size(cfg, batch, n_q) if self.fused_out else 0)
         self.ws_gemm = torch.empty(max(gemm_ws, 256), dtype=torch.uint8, device=dev)
         self.ws_decode = torch.empty(abi.mla_decode_workspace_size(cfg, batch, n_q, max_workers),
                                      dtype=torch.uint8, device=dev)
@@ -55,8 +65,24 @@ class DecodeLayer:
     def queries(self, x, pos, stream=None):
         W_DQ = self.W.get("W_DQ")
         W_UQ = self.W["W_UQ"] if "W_UQ" in self.W else self.W["W_Q"]
-        abi.mla_absorb_q(self.cfg, x, W_DQ, W_UQ, self.W["W_UK"], pos, self.q_lat, self.q_rope,
-                         self.ws_gemm, stream)
+        if self.packed:
+            abi.mla_absorb_q_packed(self.cfg, x, W_DQ, W_UQ, self.W["W_UK"], pos, self.q_packed, self.ws_gemm,
+                                    stream)
+        else:
+            abi.mla_absorb_q(self.cfg, x, W_DQ, W_UQ, self.W["W_UK"], pos, self.q_lat, self.q_rope,
+                             self.ws_gemm, stream)
+
+    def queries_fp32(self):
+        """(q_lat, q_rope) of the last step as fp32 tensors (for checks): the
+        fp32 outputs, or the packed bf16 rows (plus their remainders in
+        split-query mode) widened."""
+        if not self.packed:
+            return self.q_lat, self.q_rope
+        n = self.batch * self.n_q
+        q = self.q_packed[:n].float()
+        if self.cfg.split_query:
+            q = q + self.q_packed[n:].float()
+        return q[..., :self.cfg.d_c], q[..., self.cfg.d_c:]
 
     def append_and_queries(self, x, seq_idx, pos, stream=None):
         """The append and the query projections of one step, overlapped: the
@@ -80,25 +106,104 @@ class DecodeLayer:
             t.record_stream(self.side)
 
     def decode(self, seq_lens, stream=None):
-        abi.mla_decode(self.cfg, self.q_lat, self.q_rope, self.batch, self.n_q, self.cache, seq_lens,
-                       self.ws_decode, self.max_workers, stream)
+        if self.packed:
+            abi.mla_decode_packed(self.cfg, self.q_packed, self.batch, self.n_q, self.cache, seq_lens,
+                                  self.ws_decode, self.max_workers, stream)
+        else:
+            abi.mla_decode(self.cfg, self.q_lat, self.q_rope, self.batch, self.n_q, self.cache, seq_lens,
+                           self.ws_decode, self.max_workers, stream)
 
     def combine(self, stream=None):
         abi.mla_combine(self.cfg, self.ws_decode, self.batch, self.n_q, self.o_lat, stream)
 
     def attend(self, seq_lens, stream=None):
+        """Decode, then the latent output ``o_lat`` (merged splits, fp32)."""
         self.decode(seq_lens, stream)
         self.combine(stream)
 
-    def project(self, stream=None):
-        abi.mla_out_proj(self.cfg, self.o_lat, self.W["W_UV"], self.W["W_O"], self.y, self.ws_gemm, stream)
+    def project(self, stream=None, y=None):
+        """``y`` from this step's decode: on the bf16 path the split merge runs
+        inside the W_UV projection (``o_lat`` is not needed); otherwise from
+        ``o_lat`` (after ``combine``)."""
+        y = self.y if y is None else y
+        if self.fused_out:
+            abi.mla_combine_out_proj(self.cfg, self.ws_decode, self.batch, self.n_q, self.W["W_UV"], self.W["W_O"],
+                                     y, self.ws_gemm, self.max_workers, stream)
+        else:
+            abi.mla_out_proj(self.cfg, self.o_lat, self.W["W_UV"], self.W["W_O"], y, self.ws_gemm, stream)
 
-    def step(self, x, seq_idx, pos, seq_lens, stream=None) -> torch.Tensor:
-        """Device-resident step: returns ``y`` ``[batch * n_q, hidden]`` (a reused buffer)."""
+    def step(self, x, seq_idx, pos, seq_lens, stream=None, want_o_lat: bool = False) -> torch.Tensor:
+        """Device-resident step: returns ``y`` ``[batch * n_q, hidden]`` (a reused buffer).
+        ``want_o_lat`` also fills ``self.o_lat`` (always filled on the fp32 path)."""
         self.append_and_queries(x, seq_idx, pos, stream)
-        self.attend(seq_lens, stream)
+        self.decode(seq_lens, stream)
+        if want_o_lat or not self.fused_out:
+            self.combine(stream)
         self.project(stream)
         return self.y
+
+    def run_from_host(self, inputs, y_hosts, between=None, stream=None, copy_stream=None):
+        """Several steps over host (pinned) inputs, pipelined.
+
+        ``inputs[k]`` is ``(x, seq_idx, pos, seq_lens)`` on the host for step k;
+        step k's ``y`` lands in ``y_hosts[k]``.  The host-to-device copy of step
+        k + 1's inputs and the device-to-host copy of step k's ``y`` run on
+        ``copy_stream`` while step k computes on ``stream`` (double-buffered
+        device inputs and outputs), as a serving loop would overlap them.
+        ``between(k)``, if given, runs on ``stream`` before step k's compute.
+        Returns the host buffers; the caller synchronises."""
+        stream = stream or torch.cuda.current_stream()
+        copy_stream = copy_stream or self._copy_stream()
+        dev = self.cache.pool.device
+        n = len(inputs)
+        if n == 0:
+            return y_hosts
+        shapes = tuple((tuple(t.shape), t.dtype) for t in inputs[0])
+        if getattr(self, "_pipe_shapes", None) != shapes:   # kept across calls: work may still be in flight
+            self._pipe_bufs = ([[torch.empty_like(t, device=dev) for t in inputs[0]] for _ in range(2)],
+                               [torch.empty_like(self.y) for _ in range(2)])
+            self._pipe_shapes = shapes
+        dbuf, ybuf = self._pipe_bufs
+        copy_stream.wait_stream(stream)   # nothing of this call starts before work already queued on stream
+        loaded = [torch.cuda.Event() for _ in range(n)]
+        computed = [torch.cuda.Event() for _ in range(n)]
+        drained = [torch.cuda.Event() for _ in range(n)]
+
+        def load(k):
+            with torch.cuda.stream(copy_stream):
+                if k >= 2:   # the step that last used this input buffer has finished
+                    copy_stream.wait_event(computed[k - 2])
+                for d, h in zip(dbuf[k % 2], inputs[k]):
+                    d.copy_(h, non_blocking=True)
+                loaded[k].record(copy_stream)
+
+        load(0)
+        for k in range(n):
+            if k + 1 < n:
+                load(k + 1)
+            stream.wait_event(loaded[k])
+            if k >= 2:       # the y buffer of step k - 2 has been copied out
+                stream.wait_event(drained[k - 2])
+            if between is not None:
+                between(k)
+            x, seq_idx, pos, seq_lens = dbuf[k % 2]
+            self.append_and_queries(x, seq_idx, pos, stream)
+            self.decode(seq_lens, stream)
+            if not self.fused_out:
+                self.combine(stream)
+            self.project(stream, y=ybuf[k % 2])
+            computed[k].record(stream)
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(computed[k])
+                y_hosts[k].copy_(ybuf[k % 2], non_blocking=True)
+                drained[k].record(copy_stream)
+        stream.wait_event(drained[n - 1])
+        return y_hosts
+
+    def _copy_stream(self):
+        if getattr(self, "_copies", None) is None:
+            self._copies = torch.cuda.Stream(device=self.cache.pool.device)
+        return self._copies
 
     def step_from_host(self, x_host, seq_idx_host, pos_host, seq_lens_host, y_host,
                        stream: Optional[torch.cuda.Stream] = None):

@@ -18,15 +18,15 @@ def tol_for(shape) -> float:
     return 1e-2 if shape.dtype == "bf16" else 1e-4
 
 
-def run_gpu(wl, data=None, max_workers: int = 0, pool: Optional[torch.Tensor] = None):
+def run_gpu(wl, data=None, max_workers: int = 0, pool: Optional[torch.Tensor] = None, packed_query: bool = True):
     data = data if data is not None else generate(wl)
     dev = device_inputs(data, "cuda", pool=pool)
     cfg = Config.from_shape(wl.shape, split_query=wl.split_query)
     cache = Cache(dev["pool"], dev["block_table"])
-    layer = DecodeLayer(cfg, dev["weights"], cache, wl.batch, wl.n_q, max_workers)
+    layer = DecodeLayer(cfg, dev["weights"], cache, wl.batch, wl.n_q, max_workers, packed_query=packed_query)
     if wl.cached_from_append:
         layer.append(dev["x_cached"], dev["seq_idx_cached"], dev["pos_cached"])
-    layer.step(dev["x_new"], dev["seq_idx"], dev["pos"], dev["seq_lens"])
+    layer.step(dev["x_new"], dev["seq_idx"], dev["pos"], dev["seq_lens"], want_o_lat=True)
     torch.cuda.synchronize()
     check_device_error()
     return data, dev, layer
@@ -90,8 +90,9 @@ def check_new_cache_rows(layer, data, exp):
 def check_outputs(layer, data, exp, tokens: Iterable[int]):
     wl = data.workload
     tol = tol_for(wl.shape)
-    q_lat = oracle.to64(layer.q_lat.cpu())
-    q_rope = oracle.to64(layer.q_rope.cpu())
+    ql, qr = layer.queries_fp32()
+    q_lat = oracle.to64(ql.cpu())
+    q_rope = oracle.to64(qr.cpu())
     o_lat = layer.o_lat.cpu().double().numpy()
     y = oracle.to64(layer.y.cpu())
     worst = {}

@@ -108,6 +108,7 @@ def test_empty_work_is_a_no_op(lib):
     assert lib.mla_decode(P(c), None, None, 0, 1, None, None, 0, None, 0, None) == abi.MLA_OK
     assert lib.mla_combine(P(c), None, 0, 0, 1, None, None) == abi.MLA_OK
     assert lib.mla_out_proj(P(c), None, 0, None, None, None, None, 0, None) == abi.MLA_OK
+    assert lib.mla_combine_out_proj(P(c), None, 0, 0, 1, 0, None, None, None, None, 0, None) == abi.MLA_OK
 
 
 def test_decode_workspace_grows_with_workers_and_batch(lib):
@@ -116,7 +117,7 @@ def test_decode_workspace_grows_with_workers_and_batch(lib):
     a = lib.mla_decode_workspace_size(P(c), 64, 1, 74)
     b = lib.mla_decode_workspace_size(P(c), 64, 1, 148)
     d = lib.mla_decode_workspace_size(P(c), 64, 2, 74)
-    seg_bytes = 128 * 512 * 4
+    seg_bytes = 128 * 512 * 2     # bf16 partial output of one segment, all heads
     # one partial slot per worker and per query row
     assert b - a >= 74 * seg_bytes and d - a >= 64 * seg_bytes
 
@@ -149,3 +150,25 @@ def test_unaligned_tensors_are_rejected_on_the_bf16_path(lib):
     need = lib.mla_decode_workspace_size(P(c), 1, 1, 8)
     assert lib.mla_decode(P(c), ok, ok, 1, 1, P(cache), ok, 8, ok, need, None) == abi.MLA_ERR_INVALID_ARG
     assert lib.mla_combine(P(c), ok, need, 1, 1, bad, None) == abi.MLA_ERR_INVALID_ARG
+
+
+def test_fused_projection_checks_its_arguments(lib):
+    P = ctypes.byref
+    c = _cfg(hidden=7168, n_heads=128, d_c=512, d_r=64, qk_nope=128, v_head=128, q_lora=1536, dtype="bf16")
+    fake = ctypes.c_void_p(1 << 20)
+    need = lib.mla_combine_out_proj_workspace_size(P(c), 64, 1)
+    # W_O partials (none for 64 tokens with one K split) + the bf16 head outputs
+    assert need >= 64 * 128 * 128 * 2
+    dws = lib.mla_decode_workspace_size(P(c), 64, 1, 0)
+    assert lib.mla_combine_out_proj(P(c), None, dws, 64, 1, 0, fake, fake, fake, fake, need, None) == \
+        abi.MLA_ERR_INVALID_ARG
+    assert lib.mla_combine_out_proj(P(c), fake, dws - 256, 64, 1, 0, fake, fake, fake, fake, need, None) == \
+        abi.MLA_ERR_WORKSPACE
+    assert lib.mla_combine_out_proj(P(c), fake, dws, 64, 1, 0, fake, fake, fake, fake, need - 256, None) == \
+        abi.MLA_ERR_WORKSPACE
+    # more than 512 segments (rows + workers - 1) is not supported by the fused path
+    assert lib.mla_combine_out_proj(P(c), fake, 1 << 40, 600, 1, 0, fake, fake, fake, fake, 1 << 40, None) == \
+        abi.MLA_ERR_UNSUPPORTED
+    f32 = _cfg(dtype="f32")
+    assert lib.mla_combine_out_proj_workspace_size(P(f32), 1, 1) == 0
+

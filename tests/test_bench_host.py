@@ -67,3 +67,16 @@ def test_recorded_traffic_follows_the_decode_sources(bench, tmp_path, monkeypatc
 
 def test_rank_seeds_differ_per_rank(bench):
     assert len({bench.rank_seed(0, r) for r in range(8)}) == 8
+
+
+def test_percentiles_are_nearest_rank(bench):
+    assert bench.percentiles([]) is None
+    assert bench.percentiles([7.0]) == {"p50": 7.0, "p95": 7.0, "p99": 7.0}
+    p = bench.percentiles([float(x) for x in range(200, 0, -1)])   # order does not matter
+    assert p == {"p50": 100.0, "p95": 190.0, "p99": 198.0}
+
+
+def test_reference_arm_reports_the_gpu_arms_metric(bench):
+    import inspect
+    src = inspect.getsource(bench.run_reference) + inspect.getsource(bench.run_ours)
+    assert src.count('"metric": METRIC') == 2
