@@ -13,34 +13,49 @@
 // A worker is a cluster of two CTAs on two SMs.  CTA r owns heads
 // [64 r, 64 r + 64): its TMEM holds those heads' scores and their whole
 // 512-wide latent output.  The pages are walked two at a time (a 128-token
-// tile).  The scores of a tile are one pair MMA per 16-value K step, M = 128
-// heads (A split by heads), N = 128 tokens (B split by pages: CTA r holds
-// page r of the tile, all 576 values), so every page is read from memory
-// once and every score is computed once.  P V is a pair MMA per 16 tokens
-// and 128-column latent chunk m, N split by columns: CTA r supplies columns
-// 128 m + 64 r + (0..63), which for its own page is its score slab 2 m + r,
-// kept in place, and for the other page is that page's slab 2 m + r,
-// fetched into the slot of the other CTA's matching slab once the scores
-// have read it (an L2 hit: the other CTA has just loaded that page).  The
-// rows of D that a pair MMA leaves in one CTA's TMEM sit in 128 lanes x N/2
-// columns: lane l holds head 64 r + (l mod 64), lanes 0..63 the first half
-// of the N columns and lanes 64..127 the second.
+// tile; CTA r loads page r of the tile).
 //
-// Warp roles (224 threads per CTA): warp 0 issues the score-side TMA loads
-// and warp 6 the value-side ones (both CTAs, counted on the leader's
-// barriers); warp 1 of the leader issues every MMA of the pair; warps 2..5
+// Scores: one pair MMA per 16-value K step, M = 128 heads (A split by
+// heads), N = 128 tokens (B split by pages), so every page is read from
+// memory once and every score is computed once.
+//
+// P V: one pair MMA per 16 tokens of a page and 256-column latent block j,
+// N = 256 split by columns: CTA r supplies columns 256 j + 128 r + (0..127),
+// the slab pair m = 2 j + r (two 64-column slabs, 16 KiB).  A CTA keeps the
+// pairs of its own page that it supplies (m mod 2 = r).  Into the double
+// slot of each other pair m it fetches, once the scores have read it, the
+// other page's pair m ^ 1 (an L2 hit: the other CTA has just loaded that
+// page).  Either way the double slot of pair m feeds the P V steps of page
+// m mod 2.  The rows of D that a pair MMA leaves in one CTA's TMEM sit in
+// 128 lanes x N/2 columns: lane l holds head 64 r + (l mod 64), lanes 0..63
+// the first half of the N columns and lanes 64..127 the second.
+//
+// Barriers are per tile (a ring of 4): the value-slab loads of a tile (both
+// CTAs, 8 slabs each) complete one barrier, its score MMAs commit one, its value
+// reloads complete one and its P V commits one, so the MMA thread waits and
+// commits a few times per tile and otherwise issues MMAs back to back.
+//
+// Pipeline: the score MMAs of tile i + 1 are issued as soon as the softmax
+// of tile i has copied the scores to registers (freeing them), and P V of
+// tile i as soon as its P is written, by a second issuing warp: the tensor
+// pipe interleaves the two.  Before the softmax of tile i writes P or
+// rescales O it waits for P V of tile i - 1.
+//
+// Warp roles (256 threads per CTA, each role on whole warps with one lane
+// issuing): warp 0 issues the score-side TMA loads and warp 6 the value-side
+// ones (both CTAs, counted on the leader's barriers); in the leader, warp 1
+// issues the pair's score MMAs and warp 7 its P V MMAs; warps 2..5
 // run the online softmax, one TMEM lane per thread (a head and one page of
-// the tile), and write the segment's partial output.  Per tile the tensor
-// pipe runs the scores, then (once the softmax has written P) P V, so the
-// previous tile's P V is over when the next scores arrive.
+// the tile), and write the segment's partial output.
 //
 // TMEM (512 columns): [0,64) the score tile, [64,320) the latent output
-// (four 64-column chunks), [320,512) the query's latent columns 0..383 (A of
+// (two 128-column blocks), [320,512) the query's latent columns 0..383 (A of
 // the first 24 score K steps).
 //
 // Shared memory: the query's last 3 K slabs (64 heads x 64 values, 128-byte
-// swizzle, K-major), P (2 pages x 64 heads x 64 tokens) and a ring of 8 KiB
-// slots for page slabs (and, in split-query mode, the low query slabs).
+// swizzle, K-major), P (2 pages x 64 heads x 64 tokens), a ring of 16 KiB
+// double slots for the value slab pairs and a short ring of 8 KiB slots for
+// the rotary slab (and, in split-query mode, the low query slabs).
 //
 // The last page of a row may be partial: it is loaded with its row
 // coordinate shifted down by the missing rows, so the rows past the visible
@@ -64,34 +79,60 @@ constexpr int kH = 128, kHalfH = 64, kDc = 512, kDr = 64, kBS = 64, kRow = kDc +
 constexpr int kSlabs = kRow / 64;  // 9 K slabs of 64 values
 constexpr int kTmemQSlabs = 6;     // query K slabs held in TMEM (latent columns 0..383)
 constexpr int kSmemQSlabs = kSlabs - kTmemQSlabs;
-constexpr int kVSlabs = kDc / 64;  // 8 slabs hold latent (value) columns, the ninth the rotary key
+constexpr int kPairs = kDc / 128;  // 4 value slab pairs per page; the ninth slab is the rotary key
 constexpr int kSlab = 64 * 128;    // 64 rows x 64 bf16, 128-byte swizzle
-// Ring of 8 KiB slots (build-time tunable; the default fills the 227 KiB of
-// shared memory beside the query and P buffers).
-#ifndef MLA_PAIR_RING
-#define MLA_PAIR_RING 22
+// Double slots for value slab pairs (build-time tunable; the defaults fill
+// the shared memory beside the query, P and the short ring).
+#ifndef MLA_PAIR_VSLOTS
+#define MLA_PAIR_VSLOTS 10
 #endif
-// How far (in K slabs) the score-side loads of a tile may run ahead of the
-// previous tile's score MMAs.  The SM's TMA engine serves loads in issue
-// order, so a whole tile of score slabs issued early would queue the
-// previous tile's value reloads (needed sooner, by its P V) behind them.
-#ifndef MLA_PAIR_AHEAD
-#define MLA_PAIR_AHEAD 3
+#ifndef MLA_PAIR_VSLOTS_SPLIT
+#define MLA_PAIR_VSLOTS_SPLIT 9
 #endif
-constexpr int kRing = MLA_PAIR_RING, kAhead = MLA_PAIR_AHEAD;
 constexpr int kTmemS = 0, kTmemO = 64, kTmemQ = 320, kTmemCols = 512;
 constexpr int kSoftmaxWarps = 4;
-constexpr int kSoftmaxWarp0 = 2;                    // warps 2..5
+constexpr int kSoftmaxWarp0 = 2;  // warps 2..5
 constexpr int kVcWarp = kSoftmaxWarp0 + kSoftmaxWarps;
-constexpr int kThreads = 32 * (kVcWarp + 1);
+constexpr int kPvWarp = kVcWarp + 1;
+constexpr int kThreads = 32 * (kPvWarp + 1);
 constexpr float kRescaleLog2 = 8.f;
 constexpr uint16_t kBoth = 3;  // multicast mask: both CTAs of the pair
 
+// Ring geometry.  Value pair m of tile ti is item g = 4 ti + m of the double
+// slot ring; the short ring carries per tile the rotary slab, and in
+// split-query mode the 9 low query slabs in K order (item k = e for the low
+// slab e < 8, 8 for the rotary slab, 9 for the low slab 8).  Per-tile
+// barriers form a ring of kT.
+constexpr int kT = 4;
+__device__ __forceinline__ int tslot(int ti) { return ti % kT; }
+__device__ __forceinline__ uint32_t tpar(int ti) { return (uint32_t)(ti / kT) & 1u; }
+
+template <bool kSplit>
+struct Ring {
+  static constexpr int kV = kSplit ? MLA_PAIR_VSLOTS_SPLIT : MLA_PAIR_VSLOTS;
+  static constexpr int kS = kSplit ? 3 : 2;
+  static constexpr int kPerTile = kSplit ? kSlabs + 1 : 1;
+  static constexpr int kRope = kSplit ? 8 : 0;
+  __device__ static int vslot(int ti, int m) { return (ti * kPairs + m) % kV; }
+  __device__ static uint32_t vuse(int ti, int m) { return (uint32_t)((ti * kPairs + m) / kV); }
+  __device__ static int lo_item(int e) { return e < 2 * kPairs ? e : 9; }
+  __device__ static int sslot(int ti, int k) { return (ti * kPerTile + k) % kS; }
+  __device__ static uint32_t suse(int ti, int k) { return (uint32_t)((ti * kPerTile + k) / kS); }
+};
+
+// A tile's value pairs may reuse only double slots whose P V was issued before
+// the tile's scores (P V runs one tile behind): at least two tiles of slots.
+static_assert(Ring<false>::kV >= 2 * kPairs && Ring<true>::kV >= 2 * kPairs, "too few double slots");
+
+template <bool kSplit>
 struct Smem {
+  using R = Ring<kSplit>;
   uint8_t q[kSmemQSlabs][kSlab];  // query K slabs 6..8; first member: 1024-byte aligned
   uint8_t p[2][kSlab];            // P of the tile: [page of the tile] 64 heads x 64 tokens
-  uint8_t ring[kRing][kSlab];     // page slabs (and low query slabs)
-  uint64_t full[kRing], qkd[kRing], vfull[kRing], empty[kRing];
+  uint8_t v[R::kV][2][kSlab];     // value slab pairs (score-side B, then P V B)
+  uint8_t r[R::kS][kSlab];        // rotary slabs (and low query slabs)
+  uint64_t kfull[kT], qkd[kT], vfull[kT], vempty[kT];  // per tile: score loads, score MMAs, reloads, P V
+  uint64_t rfull[R::kS], rempty[R::kS];                 // short ring
   uint64_t q_full, q_empty, qt_full;
   uint64_t s_full, s_free, p_full, pv_done;
   uint64_t o_free, fin, xbar[2], lbar;
@@ -101,22 +142,32 @@ struct Smem {
   int abort_flag;
 };
 
-constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
-static_assert(kSmemBytes <= 232448, "shared memory over the 227 KiB per-block limit");
+template <bool kSplit>
+constexpr size_t smem_bytes() {
+  return sizeof(Smem<kSplit>) + 1024;
+}
+static_assert(smem_bytes<false>() <= 232448, "shared memory over the 227 KiB per-block limit");
+static_assert(smem_bytes<true>() <= 232448, "shared memory over the 227 KiB per-block limit");
 
 struct Params {
   const bf16* q;  // packed query rows [rows][H][576] (the TMEM part is read from here)
   const int32_t* block_table;
   const int32_t* seq_lens;
-  int max_blocks, num_blocks, n_q, split;
+  int max_blocks, num_blocks, n_q;
   float scale_log2;
   unsigned long long wait_ns;
   void* ws;
   DecodeLayout L;
 };
 
-__device__ __forceinline__ void set_abort(Smem& sm) { *(volatile int*)&sm.abort_flag = 1; }
-__device__ __forceinline__ bool aborted(Smem& sm) { return *(volatile int*)&sm.abort_flag != 0; }
+template <bool kSplit>
+__device__ __forceinline__ void set_abort(Smem<kSplit>& sm) {
+  *(volatile int*)&sm.abort_flag = 1;
+}
+template <bool kSplit>
+__device__ __forceinline__ bool aborted(Smem<kSplit>& sm) {
+  return *(volatile int*)&sm.abort_flag != 0;
+}
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -134,21 +185,59 @@ __device__ __forceinline__ uint64_t kmajor_desc(const void* p, uint32_t byte_off
 // Descriptors differ only in the start address (bits 0-13, 16-byte units).
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t byte_offset) { return d + (byte_offset >> 4); }
 
+// ---------------------------------------------------------------- warp-uniform roles
+// Every role runs on whole warps; one lane issues the TMA, MMA, commit and
+// expect-tx instructions.  Values that all lanes hold alike are broadcast
+// from lane 0 (uni), so that they and the descriptors and coordinates built
+// from them stay in the warp-uniform datapath those instructions read from
+// (a value the compiler must treat as per-lane costs a slow move into it at
+// every instruction whose operands changed).
+__device__ __forceinline__ int uni(int x) { return __shfl_sync(0xffffffffu, x, 0); }
+
+#ifndef MLA_SOFTMAX_SLEEP_NS
+#define MLA_SOFTMAX_SLEEP_NS 0
+#endif
+// A warp waits with lane 0 polling while the others sit at the warp barrier
+// (waiting warps do not flood the SM's shared-memory pipe); the outcome is
+// the warp's.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int where, uint64_t wns, int lane,
+                                          uint32_t sleep_ns = 0) {
+  int ok = 1;
+  if (lane == 0) ok = mbar_wait(bar, parity, where, wns, sleep_ns) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
 // ---------------------------------------------------------------- tiles
-// Walks the worker's tiles in order: segment, first page of the tile.
+// Walks the worker's tiles in order: segment, first page of the tile (whole
+// warps only: the segment is read once and broadcast).
 struct Tiles {
   const int4* segs;
   int si, seg_end, pg, nseg;  // nseg: segments started so far (this one included)
-  __device__ Tiles(const int4* s, int b, int e) : segs(s), si(b), seg_end(e), pg(b < e ? s[b].y : 0), nseg(1) {}
+  int v, pg0, pg1;            // the segment: query row, first page, end page
+  __device__ Tiles(const int4* s, int b, int e) : segs(s), si(b), seg_end(e), pg(0), nseg(1), v(0), pg0(0), pg1(0) {
+    load();
+    pg = pg0;
+  }
+  __device__ void load() {
+    if (si < seg_end) {
+      const int4 g = segs[si];
+      v = uni(g.x);
+      pg0 = uni(g.y);
+      pg1 = uni(g.z);
+    }
+  }
   __device__ bool valid() const { return si < seg_end; }
-  __device__ int4 seg() const { return segs[si]; }
-  __device__ bool first() const { return pg == segs[si].y; }
-  __device__ bool last() const { return pg + 2 >= segs[si].z; }
-  __device__ bool has_b() const { return pg + 1 < segs[si].z; }
+  __device__ int row() const { return v; }
+  __device__ bool first() const { return pg == pg0; }
+  __device__ bool last() const { return pg + 2 >= pg1; }
+  __device__ bool has_b() const { return pg + 1 < pg1; }
   __device__ void next() {
     pg += 2;
-    if (pg >= segs[si].z && ++si < seg_end) {
-      pg = segs[si].y;
+    if (pg >= pg1 && ++si < seg_end) {
+      load();
+      pg = pg0;
       ++nseg;
     }
   }
@@ -172,86 +261,105 @@ __device__ __forceinline__ int phys_block(const Params& p, int v, int blk, bool 
   return phys;
 }
 
-// ---------------------------------------------------------------- ring items
-// Per tile every role walks the same item sequence: for K slab e = 0..8 a
-// page item (this CTA's page slab e), followed in split-query mode by a low
-// query item (the slab e of the query's bf16 remainder).  Item n lives in
-// ring slot n mod kRing.  A page item with e < 8 is kept until the tile's
-// P V: one CTA of the pair keeps its own slab, the other replaces its slab,
-// once the scores have read it, by the matching value slab of the other page
-// (see the header comment); the rotary slab and low query items are freed
-// right after the scores.
-struct Items {
-  int per_tile;
-  __device__ explicit Items(int split) : per_tile(split ? 2 * kSlabs : kSlabs) {}
-  __device__ uint32_t page(int tile, int e) const { return (uint32_t)(tile * per_tile + e * (per_tile / kSlabs)); }
-};
-
-// Per-slot use counters of the barriers that not every item uses.
-struct SlotUses {
-  uint8_t n[kRing];
-  __device__ SlotUses() {
-    for (int i = 0; i < kRing; ++i) n[i] = 0;
-  }
-  __device__ uint32_t next(int slot) { return n[slot]++ & 1u; }
-};
-
-// Which CTA of the pair fetches the other page's half for value slab e, and
-// which slab of which page of the tile that is: for even e = 2m CTA 1 needs
-// page 0's slab 2m + 1; for odd e = 2m + 1 CTA 0 needs page 1's slab 2m.
-__device__ __forceinline__ uint32_t reloader(int e) { return (e & 1) ? 0u : 1u; }
-__device__ __forceinline__ int reload_page(int e) { return (e & 1) ? 1 : 0; }
-__device__ __forceinline__ int reload_slab(int e) { return (e & 1) ? e - 1 : e + 1; }
-
 // ---------------------------------------------------------------- TMA producers
 // Score-side loads (warp 0): the segment's query slabs held in shared
-// memory, then per tile the 9 slabs of this CTA's page (and the low query
-// slabs), each into the next ring slot once its previous use is over.
-__device__ void producer_k(Smem& sm, const CUtensorMap* pool, const CUtensorMap* qmap, const CUtensorMap* qlomap,
-                           const Params& p, int seg_begin, int seg_end, uint32_t rank) {
+// memory, then per tile the 8 value slabs of this CTA's page into their
+// pairs' double slots (counted on the tile's barrier), then the short-ring
+// items: the rotary slab and, in split-query mode, the low query slabs (one
+// barrier each).
+template <bool kSplit>
+__device__ void producer_k(Smem<kSplit>& sm, const CUtensorMap* pool, const CUtensorMap* qmap,
+                           const CUtensorMap* qlomap, const Params& p, int seg_begin, int seg_end, uint32_t rank,
+                           int lane) {
+  using R = Ring<kSplit>;
   const int4* segs = ws_at<int4>(p.ws, p.L.off_seg);
-  const bool lead = rank == 0;
-  const Items items(p.split);
-  SlotUses qkd_use;
-  uint32_t n = 0;  // items issued
-  int nq = 0;      // query loads issued
+  const bool lead = rank == 0, issue = lane == 0;
+  const uint64_t wns = p.wait_ns;
+  int nq = 0;  // query loads issued
   int ti = 0;
-  for (Tiles t(segs, seg_begin, seg_end); t.valid() && !aborted(sm); t.next(), ++ti) {
-    // phases of the previous tile's "scores have read value slab e" barriers
-    uint32_t prev_qkd[kVSlabs];
-    if (ti >= 1)
-      for (int e = 0; e < kVSlabs; ++e) prev_qkd[e] = qkd_use.next((int)(items.page(ti - 1, e) % kRing));
-    const int v = t.seg().x;
+  for (Tiles t(segs, seg_begin, seg_end); t.valid() && !uni(aborted(sm) ? 1 : 0); t.next(), ++ti) {
+    const int v = t.row();
     if (t.first()) {
-      if (nq >= 1 && !mbar_wait(&sm.q_empty, (nq - 1) & 1, 70, p.wait_ns)) goto fail;
-      if (lead) mbar_arrive_expect_tx(&sm.q_full, 2 * kSmemQSlabs * kSlab);
-      for (int e = kTmemQSlabs; e < kSlabs; ++e)
-        tma_load_2d_pair(sm.q[e - kTmemQSlabs], qmap, 64 * e, v * kH + kHalfH * (int)rank, leader(&sm.q_full));
+      if (nq >= 1 && !warp_wait(&sm.q_empty, (nq - 1) & 1, 70, wns, lane)) goto fail;
+      if (issue) {
+        if (lead) mbar_arrive_expect_tx(&sm.q_full, 2 * kSmemQSlabs * kSlab);
+        for (int e = kTmemQSlabs; e < kSlabs; ++e)
+          tma_load_2d_pair(sm.q[e - kTmemQSlabs], qmap, 64 * e, v * kH + kHalfH * (int)rank, leader(&sm.q_full));
+      }
       ++nq;
     }
     const bool has = rank == 0 || t.has_b();
     const int blk = t.pg + (int)rank;
-    const int phys = has ? phys_block(p, v, blk, true) : 0;
-    const int y = has ? page_valid(visible_len(p, v), blk) - kBS : 0;
+    const int phys = has ? uni(phys_block(p, v, blk, true)) : 0;
+    const int y = has ? uni(page_valid(visible_len(p, v), blk) - kBS) : 0;
     const uint32_t page_bytes = (t.has_b() ? 2 : 1) * kSlab;
-    for (int e = 0; e < kSlabs; ++e) {
-      if (ti >= 1) {  // pace: the previous tile's scores have read slab e + kAhead
-        const int ea = e + kAhead;
-        const bool ok = ea < kVSlabs
-                            ? mbar_wait(&sm.qkd[items.page(ti - 1, ea) % kRing], prev_qkd[ea], 74, p.wait_ns)
-                            : mbar_wait(&sm.s_full, (ti - 1) & 1, 75, p.wait_ns);
-        if (!ok) goto fail;
+    // without split-query low slabs the short ring holds only rotary slabs: load it first
+    if (!kSplit) {
+      const int sl = R::sslot(ti, R::kRope);
+      const uint32_t use = R::suse(ti, R::kRope);
+      if (use >= 1 && !warp_wait(&sm.rempty[sl], (use - 1) & 1, 72, wns, lane)) goto fail;
+      if (issue && lead) mbar_arrive_expect_tx(&sm.rfull[sl], page_bytes);
+      if (issue && has) tma_load_3d_pair(sm.r[sl], pool, 64 * (kSlabs - 1), y, phys, leader(&sm.rfull[sl]));
+    }
+    // the tile barrier's previous phase (tile ti - kT) is over once that tile's scores were issued
+    if (ti >= kT && !warp_wait(&sm.qkd[tslot(ti)], tpar(ti - kT), 69, wns, lane)) goto fail;
+    if (issue && lead) mbar_arrive_expect_tx(&sm.kfull[tslot(ti)], 2 * kPairs * page_bytes);
+    for (int e = 0; e < 2 * kPairs; ++e) {  // the 8 value slabs, on the tile barrier
+      const int g = ti * kPairs + (e >> 1);
+      if ((e & 1) == 0 && g >= R::kV) {  // the double slot's previous tile is past its P V
+        const int tp = (g - R::kV) / kPairs;
+        if (!warp_wait(&sm.vempty[tslot(tp)], tpar(tp), 71, wns, lane)) goto fail;
       }
-      for (int lo = 0; lo <= p.split; ++lo, ++n) {
-        const int slot = (int)(n % kRing);
-        const uint32_t use = n / kRing;
-        if (use >= 1 && !mbar_wait(&sm.empty[slot], (use - 1) & 1, 71, p.wait_ns)) goto fail;
-        if (lo == 0) {
-          if (lead) mbar_arrive_expect_tx(&sm.full[slot], page_bytes);
-          if (has) tma_load_3d_pair(sm.ring[slot], pool, 64 * e, y, phys, leader(&sm.full[slot]));
-        } else {  // the low part of the query for the same K slab
-          if (lead) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlab);
-          tma_load_2d_pair(sm.ring[slot], qlomap, 64 * e, v * kH + kHalfH * (int)rank, leader(&sm.full[slot]));
+      if (issue && has)
+        tma_load_3d_pair(sm.v[g % R::kV][e & 1], pool, 64 * e, y, phys, leader(&sm.kfull[tslot(ti)]));
+    }
+    // then (split-query mode) the short-ring items in their order (the score MMAs free them one by one)
+    for (int k = 0; kSplit && k < R::kPerTile; ++k) {
+      const int sl = R::sslot(ti, k);
+      const uint32_t use = R::suse(ti, k);
+      if (use >= 1 && !warp_wait(&sm.rempty[sl], (use - 1) & 1, 72, wns, lane)) goto fail;
+      if (!issue) continue;
+      if (k == R::kRope) {
+        if (lead) mbar_arrive_expect_tx(&sm.rfull[sl], page_bytes);
+        if (has) tma_load_3d_pair(sm.r[sl], pool, 64 * (kSlabs - 1), y, phys, leader(&sm.rfull[sl]));
+      } else {  // the low part of the query for K slab e
+        const int e = k < 2 * kPairs ? k : kSlabs - 1;
+        if (lead) mbar_arrive_expect_tx(&sm.rfull[sl], 2 * kSlab);
+        tma_load_2d_pair(sm.r[sl], qlomap, 64 * e, v * kH + kHalfH * (int)rank, leader(&sm.rfull[sl]));
+      }
+    }
+  }
+  return;
+fail:
+  set_abort(sm);
+}
+
+// Value-side loads (warp 6): once the scores of a tile have been computed,
+// for every pair m the CTA that does not supply pair m's columns fetches the
+// other page's pair m ^ 1 into that double slot; the leader counts the
+// tile's bytes on one barrier.
+template <bool kSplit>
+__device__ void producer_v(Smem<kSplit>& sm, const CUtensorMap* pool, const Params& p, int seg_begin, int seg_end,
+                           uint32_t rank, int lane) {
+  using R = Ring<kSplit>;
+  const int4* segs = ws_at<int4>(p.ws, p.L.off_seg);
+  const bool lead = rank == 0, issue = lane == 0;
+  int ti = 0;
+  for (Tiles t(segs, seg_begin, seg_end); t.valid() && !uni(aborted(sm) ? 1 : 0); t.next(), ++ti) {
+    const int v = t.row(), len_v = uni(visible_len(p, v));
+    if (!warp_wait(&sm.qkd[tslot(ti)], tpar(ti), 73, p.wait_ns, lane)) goto fail;
+    // pairs 0 and 2 read page 0, pairs 1 and 3 page 1 (absent in a one-page tile)
+    if (issue && lead) mbar_arrive_expect_tx(&sm.vfull[tslot(ti)], (t.has_b() ? 4 : 2) * 2 * kSlab);
+    // this CTA reloads the pairs m with m mod 2 != rank, all from page 1 - rank
+    const int pgi = 1 - (int)rank;
+    if (pgi == 0 || t.has_b()) {
+      const int blk = t.pg + pgi;
+      const int y = page_valid(len_v, blk) - kBS, phys = uni(phys_block(p, v, blk, false));
+      for (int m = pgi; m < kPairs; m += 2) {
+        const int ds = R::vslot(ti, m), x = 128 * (m ^ 1);
+        if (issue) {
+          tma_load_3d_pair(sm.v[ds][0], pool, x, y, phys, leader(&sm.vfull[tslot(ti)]));
+          tma_load_3d_pair(sm.v[ds][1], pool, x + 64, y, phys, leader(&sm.vfull[tslot(ti)]));
         }
       }
     }
@@ -261,127 +369,150 @@ fail:
   set_abort(sm);
 }
 
-// Value-side loads (warp 6): once the scores have read value slab e of a
-// tile, the CTA that does not keep it fetches the other page's matching slab
-// into the same slot (it is in L2: the other CTA loaded that page for its
-// scores); the leader counts the bytes.
-__device__ void producer_v(Smem& sm, const CUtensorMap* pool, const Params& p, int seg_begin, int seg_end,
-                           uint32_t rank) {
-  const int4* segs = ws_at<int4>(p.ws, p.L.off_seg);
-  const bool lead = rank == 0;
-  const Items items(p.split);
-  SlotUses qkd_use;
-  int ti = 0;
-  for (Tiles t(segs, seg_begin, seg_end); t.valid() && !aborted(sm); t.next(), ++ti) {
-    const int v = t.seg().x, len_v = visible_len(p, v);
-    for (int e = 0; e < kVSlabs; ++e) {
-      const int slot = (int)(items.page(ti, e) % kRing);
-      if (!mbar_wait(&sm.qkd[slot], qkd_use.next(slot), 73, p.wait_ns)) goto fail;
-      const int pgi = reload_page(e);
-      const bool exists = pgi == 0 || t.has_b();
-      if (lead) mbar_arrive_expect_tx(&sm.vfull[slot], exists ? kSlab : 0);
-      if (exists && rank == reloader(e)) {
-        const int blk = t.pg + pgi;
-        tma_load_3d_pair(sm.ring[slot], pool, 64 * reload_slab(e), page_valid(len_v, blk) - kBS,
-                         phys_block(p, v, blk, false), leader(&sm.vfull[slot]));
+// ---------------------------------------------------------------- MMA issuer (leader CTA)
+// The score MMAs of tile ti over the 9 K slabs.
+template <bool kSplit>
+__device__ bool issue_scores(Smem<kSplit>& sm, uint32_t tmem, const Tiles& t, int ti, uint64_t wns, int lane) {
+  using R = Ring<kSplit>;
+  constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+  const bool issue = lane == 0;
+  const uint32_t d = tmem + kTmemS;
+  const int rope_sl = R::sslot(ti, R::kRope);
+  // every descriptor of the tile before the waits: the MMA queue is short,
+  // so arithmetic between two MMAs would leave the tensor pipe idle
+  uint64_t bdesc[kSlabs];
+#pragma unroll
+  for (int m = 0; m < kPairs; ++m) {
+    const uint64_t b0 = kmajor_desc(sm.v[R::vslot(ti, m)][0], 0);
+    bdesc[2 * m] = b0;
+    bdesc[2 * m + 1] = desc_add(b0, kSlab);
+  }
+  bdesc[kSlabs - 1] = kmajor_desc(sm.r[rope_sl], 0);
+  const uint64_t qdesc = kmajor_desc(sm.q[0], 0);
+  if (t.first() && (!warp_wait(&sm.q_full, (t.nseg - 1) & 1, 80, wns, lane) ||
+                    !warp_wait(&sm.qt_full, (t.nseg - 1) & 1, 79, wns, lane)))
+    return false;
+  if (ti >= 1 && !warp_wait(&sm.s_free, (ti - 1) & 1, 81, wns, lane)) return false;
+  if (!warp_wait(&sm.kfull[tslot(ti)], tpar(ti), 82, wns, lane)) return false;
+  tc_fence_after();
+#pragma unroll
+  for (int e = 0; e < kSlabs; ++e) {
+    if (e == kSlabs - 1) {
+      if (!warp_wait(&sm.rfull[rope_sl], R::suse(ti, R::kRope) & 1, 78, wns, lane)) return false;
+      tc_fence_after();
+    }
+    const uint64_t bd = bdesc[e];
+    if (e < kTmemQSlabs) {  // A (query) from TMEM: 8 columns of bf16 pairs per 16-value K step
+      if (issue) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mma_ts_pair(d, tmem + kTmemQ + 32 * e + 8 * j, desc_add(bd, 32 * j), idesc_s, (e | j) ? 1u : 0u);
+      }
+    } else {
+      const uint64_t ad = desc_add(qdesc, (e - kTmemQSlabs) * kSlab);
+      if (issue) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mma_ss_pair(d, desc_add(ad, 32 * j), desc_add(bd, 32 * j), idesc_s, 1u);
+      }
+    }
+    if (kSplit) {
+      const int k = R::lo_item(e), lo_sl = R::sslot(ti, k);
+      if (!warp_wait(&sm.rfull[lo_sl], R::suse(ti, k) & 1, 83, wns, lane)) return false;
+      tc_fence_after();
+      const uint64_t ad = kmajor_desc(sm.r[lo_sl], 0);
+      if (issue) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mma_ss_pair(d, desc_add(ad, 32 * j), desc_add(bd, 32 * j), idesc_s, 1u);
+        mma_commit_pair(&sm.rempty[lo_sl], kBoth);
       }
     }
   }
-  return;
-fail:
-  set_abort(sm);
-}
-
-// ---------------------------------------------------------------- MMA issuer (leader CTA)
-// Per tile: the score MMAs over the 9 K slabs, then (after the softmax has
-// written P) P V, one 128-column latent chunk m at a time: its page-0 half
-// from value slab item 2m, its page-1 half from item 2m + 1.
-__device__ void mma_issuer(Smem& sm, uint32_t tmem, const Params& p, int seg_begin, int seg_end) {
-  const int4* segs = ws_at<int4>(p.ws, p.L.off_seg);
-  constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
-  constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, 0, 1);
-  const uint64_t wns = p.wait_ns;
-  const Items items(p.split);
-  SlotUses vfull_use;
-  int ti = 0;
-  for (Tiles t(segs, seg_begin, seg_end); t.valid(); t.next(), ++ti) {
-    // ---- scores
-    if (t.first() && (!mbar_wait(&sm.q_full, (t.nseg - 1) & 1, 80, wns) ||
-                      !mbar_wait(&sm.qt_full, (t.nseg - 1) & 1, 79, wns)))
-      goto fail;
-    if (ti >= 1 && !mbar_wait(&sm.s_free, (ti - 1) & 1, 81, wns)) goto fail;
-    tc_fence_after();
-    for (int e = 0; e < kSlabs; ++e) {
-      const uint32_t n = items.page(ti, e);
-      const int slot = (int)(n % kRing);
-      if (!mbar_wait(&sm.full[slot], (n / kRing) & 1, 82, wns)) goto fail;
-      int lo_slot = 0;
-      if (p.split) {
-        lo_slot = (int)((n + 1) % kRing);
-        if (!mbar_wait(&sm.full[lo_slot], ((n + 1) / kRing) & 1, 83, wns)) goto fail;
-      }
-      tc_fence_after();
-      const uint32_t d = tmem + kTmemS;
-      if (e < kTmemQSlabs) {  // A (query) from TMEM: 8 columns of bf16 pairs per 16-value K step
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          mma_ts_pair(d, tmem + kTmemQ + 32 * e + 8 * j, kmajor_desc(sm.ring[slot], 32 * j), idesc_s,
-                      (e | j) ? 1u : 0u);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          mma_ss_pair(d, kmajor_desc(sm.q[e - kTmemQSlabs], 32 * j), kmajor_desc(sm.ring[slot], 32 * j), idesc_s, 1u);
-      }
-      if (p.split) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          mma_ss_pair(d, kmajor_desc(sm.ring[lo_slot], 32 * j), kmajor_desc(sm.ring[slot], 32 * j), idesc_s, 1u);
-        mma_commit_pair(&sm.empty[lo_slot], kBoth);
-      }
-      mma_commit_pair(e < kVSlabs ? &sm.qkd[slot] : &sm.empty[slot], kBoth);
-    }
+  if (issue) {
+    mma_commit_pair(&sm.qkd[tslot(ti)], kBoth);
+    mma_commit_pair(&sm.rempty[rope_sl], kBoth);
     mma_commit_pair(&sm.s_full, kBoth);
     if (t.last()) mma_commit_pair(&sm.q_empty, kBoth);
+  }
+  __syncwarp();
+  return true;
+}
 
-    // ---- P V
-    if (t.first() && t.nseg >= 2 && !mbar_wait(&sm.o_free, (t.nseg - 2) & 1, 84, wns)) goto fail;
-    if (!mbar_wait(&sm.p_full, ti & 1, 85, wns)) goto fail;
-    tc_fence_after();
-    for (int e = 0; e < kVSlabs; ++e) {
-      const int m = e >> 1, pgi = e & 1;
-      const int slot = (int)(items.page(ti, e) % kRing);
-      if (!mbar_wait(&sm.vfull[slot], vfull_use.next(slot), 86, wns)) goto fail;
-      if (pgi == 0 || t.has_b()) {
-        tc_fence_after();
-        // value slab as an MN-major B operand: 64 latent columns, 8-token
-        // groups 1 KiB apart (SBO), 16 tokens per K step
-        const uint64_t vd = smem_desc(smem_u32(sm.ring[slot]), kSlab, 1024, kSwizzle128B);
+// P V of tile ti: latent block j, page q from the double slot of pair 2 j + q.
+template <bool kSplit>
+__device__ bool issue_pv(Smem<kSplit>& sm, uint32_t tmem, const Tiles& t, int ti, uint64_t wns, int lane) {
+  using R = Ring<kSplit>;
+  constexpr uint32_t idesc_o = idesc_bf16_f32(128, 256, 0, 1);
+  const bool issue = lane == 0;
+  const bool two = t.has_b(), first = t.first();
+  // the slab pairs as MN-major B operands: two 64-column groups one slab
+  // apart (LBO), 8-token groups 1 KiB apart (SBO), 16 tokens per K step
+  uint64_t vdesc[kPairs];
+#pragma unroll
+  for (int m = 0; m < kPairs; ++m) vdesc[m] = smem_desc(smem_u32(sm.v[R::vslot(ti, m)][0]), kSlab, 1024, kSwizzle128B);
+  const uint64_t pdesc = kmajor_desc(sm.p[0], 0);
+  if (first && t.nseg >= 2 && !warp_wait(&sm.o_free, (t.nseg - 2) & 1, 84, wns, lane)) return false;
+  if (!warp_wait(&sm.p_full, ti & 1, 85, wns, lane)) return false;
+  if (!warp_wait(&sm.vfull[tslot(ti)], tpar(ti), 86, wns, lane)) return false;
+  tc_fence_after();
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      if (issue && (q == 0 || two)) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss_pair(tmem + kTmemO + 64 * m, kmajor_desc(sm.p[pgi], 32 * kk), desc_add(vd, 2048 * kk), idesc_o,
-                      (t.first() && pgi == 0 && kk == 0) ? 0u : 1u);
+          mma_ss_pair(tmem + kTmemO + 128 * j, desc_add(pdesc, q * kSlab + 32 * kk), desc_add(vdesc[2 * j + q], 2048 * kk),
+                      idesc_o, (first && q == 0 && kk == 0) ? 0u : 1u);
       }
-      mma_commit_pair(&sm.empty[slot], kBoth);
     }
+  }
+  if (issue) {
+    mma_commit_pair(&sm.vempty[tslot(ti)], kBoth);
     mma_commit_pair(&sm.pv_done, kBoth);
   }
-  mma_commit_pair(&sm.fin, 1);
-  mbar_wait(&sm.fin, 0, 87, wns);
-  return;
-fail:
-  set_abort(sm);
-  mma_commit_pair(&sm.fin, 1);
-  mbar_wait(&sm.fin, 0, 88, wns);
+  __syncwarp();
+  return true;
+}
+
+// The two MMA issuers of the pair (leader CTA): warp 1 issues the scores of
+// every tile, warp 7 the P V of every tile as soon as its P is written, so
+// that the tensor pipe interleaves the two streams (P V of tile i runs among
+// the scores of tile i + 1) and neither stream's waits stall the other.  A
+// commit tracks the MMAs of the thread that issues it, so each stream's
+// barriers see only its own MMAs.  Both end on `fin` (count 2).
+template <bool kSplit>
+__device__ void score_issuer(Smem<kSplit>& sm, uint32_t tmem, const Params& p, int seg_begin, int seg_end, int lane) {
+  const int4* segs = ws_at<int4>(p.ws, p.L.off_seg);
+  const uint64_t wns = p.wait_ns;
+  int ti = 0;
+  bool ok = true;
+  for (Tiles t(segs, seg_begin, seg_end); t.valid() && ok; t.next(), ++ti) ok = issue_scores(sm, tmem, t, ti, wns, lane);
+  if (!ok) set_abort(sm);
+  if (lane == 0) mma_commit_pair(&sm.fin, 1);
+  warp_wait(&sm.fin, 0, 87, wns, lane);
+}
+
+template <bool kSplit>
+__device__ void pv_issuer(Smem<kSplit>& sm, uint32_t tmem, const Params& p, int seg_begin, int seg_end, int lane) {
+  const int4* segs = ws_at<int4>(p.ws, p.L.off_seg);
+  const uint64_t wns = p.wait_ns;
+  int ti = 0;
+  bool ok = true;
+  for (Tiles t(segs, seg_begin, seg_end); t.valid() && ok; t.next(), ++ti) ok = issue_pv(sm, tmem, t, ti, wns, lane);
+  if (!ok) set_abort(sm);
+  if (lane == 0) mma_commit_pair(&sm.fin, 1);
+  warp_wait(&sm.fin, 0, 88, wns, lane);
 }
 
 // ---------------------------------------------------------------- softmax
-#define MLA_WARP_WAIT(expr) (__all_sync(0xffffffffu, (expr)))
 
 // The query's latent columns 0..383 of this lane's head into TMEM (the A
 // operand of the first 24 score K steps).  A pair MMA with A in TMEM reads
 // each CTA's 64 rows from lanes 0..63 and again from lanes 64..127, so lanes
 // l and l ^ 64 both hold head 64 r + (l mod 64).  Then the leader is told.
-__device__ __forceinline__ void load_query_tmem(Smem& sm, const Params& p, int v, int head, uint32_t tl, int lane) {
+template <bool kSplit>
+__device__ __forceinline__ void load_query_tmem(Smem<kSplit>& sm, const Params& p, int v, int head, uint32_t tl,
+                                                int lane) {
   const uint4* src = reinterpret_cast<const uint4*>(p.q + ((long long)v * kH + head) * kRow);
 #pragma unroll 1
   for (int b = 0; b < kTmemQSlabs / 2; ++b) {  // 16 loads in flight per round, 64 columns each
@@ -403,12 +534,13 @@ __device__ __forceinline__ void load_query_tmem(Smem& sm, const Params& p, int v
   if (lane == 0) mbar_arrive_remote(leader(&sm.qt_full));
 }
 
-__device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_begin, int seg_end, uint32_t rank,
-                             int warp, int lane) {
+template <bool kSplit>
+__device__ void softmax_role(Smem<kSplit>& sm, uint32_t tmem, const Params& p, int seg_begin, int seg_end,
+                             uint32_t rank, int warp, int lane) {
   const int4* segs = ws_at<int4>(p.ws, p.L.off_seg);
   const int qw = warp & 3;                                 // TMEM lane quarter
   const int l = qw * 32 + lane;                            // TMEM lane
-  const int half = l >> 6;                                 // page of the tile / latent half of O
+  const int half = l >> 6;                                 // page of the tile / column half of each O block
   const int hl = l & 63, head = kHalfH * (int)rank + hl;   // head of this lane
   const uint32_t tl = tmem + ((uint32_t)(qw * 32) << 16);  // this warp's lane quarter
   const uint64_t wns = p.wait_ns;
@@ -418,16 +550,15 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
   float m_used = -INFINITY, lsum = 0.f;
   int nseg_done = 0;
   Tiles t(segs, seg_begin, seg_end);
-  if (t.valid()) load_query_tmem(sm, p, t.seg().x, head, tl, lane);
+  if (t.valid()) load_query_tmem(sm, p, t.row(), head, tl, lane);
   for (int i = 0; t.valid(); ++i, t.next()) {
-    const int4 sg = t.seg();
-    const int v = sg.x, len_v = visible_len(p, v);
+    const int v = t.row(), len_v = visible_len(p, v);
     const bool first = t.first(), last = t.last();
     if (first) {
       m_used = -INFINITY;
       lsum = 0.f;
     }
-    if (!MLA_WARP_WAIT(mbar_wait(&sm.s_full, i & 1, 90, wns))) goto fail;
+    if (!warp_wait(&sm.s_full, i & 1, 90, wns, lane, MLA_SOFTMAX_SLEEP_NS)) goto fail;
     tc_fence_after();
     float s[64];
     {
@@ -461,7 +592,7 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
     sm.xm[i & 1][l] = m_loc;
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.xbar[i & 1]);
-    if (!MLA_WARP_WAIT(mbar_wait(&sm.xbar[i & 1], (i >> 1) & 1, 91, wns))) goto fail;
+    if (!warp_wait(&sm.xbar[i & 1], (i >> 1) & 1, 91, wns, lane)) goto fail;
     const float m_tile = fmaxf(m_loc, sm.xm[i & 1][l ^ 64]);
 
     bool rescale = false;
@@ -484,9 +615,11 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
     }
     lsum = lsum * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
 
-    // O holds every earlier tile (their P V ran before this tile's scores on
-    // the in-order tensor pipe).  tcgen05.ld / st are warp-collective: the
-    // warp rescales when any lane needs it.
+    // P V of the previous tile reads P and accumulates into O: both must be
+    // over before this tile rescales O or overwrites P.
+    if (i >= 1 && !warp_wait(&sm.pv_done, (i - 1) & 1, 92, wns, lane)) goto fail;
+    tc_fence_after();
+    // tcgen05.ld / st are warp-collective: the warp rescales when any lane needs it.
     if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
@@ -501,8 +634,7 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
       tmem_wait_st();
     }
     {
-      // row hl of this page's P slab, K-major with the 128-byte swizzle (the
-      // previous tile's P V is over: this tile's scores ran after it)
+      // row hl of this page's P slab, K-major with the 128-byte swizzle
       uint8_t* row = sm.p[half] + hl * 128;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
@@ -515,8 +647,7 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
     if (lane == 0) mbar_arrive_remote(leader(&sm.p_full));
 
     // The scores of this segment are all done (s_full of its last tile): the
-    // next segment's query can replace this one in TMEM, before the epilogue,
-    // which waits for this tile's P V (queued before the next segment's scores).
+    // next segment's query can replace this one in TMEM before the epilogue.
     if (last && t.si + 1 < seg_end) load_query_tmem(sm, p, segs[t.si + 1].x, head, tl, lane);
 
     if (last) {
@@ -524,20 +655,20 @@ __device__ void softmax_role(Smem& sm, uint32_t tmem, const Params& p, int seg_b
       sm.xl[l] = lsum;
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.lbar);
-      if (!MLA_WARP_WAIT(mbar_wait(&sm.lbar, nseg_done & 1, 94, wns))) goto fail;
+      if (!warp_wait(&sm.lbar, nseg_done & 1, 94, wns, lane)) goto fail;
       const float ltot = lsum + sm.xl[l ^ 64];
-      if (!MLA_WARP_WAIT(mbar_wait(&sm.pv_done, i & 1, 95, wns))) goto fail;
+      if (!warp_wait(&sm.pv_done, i & 1, 95, wns, lane)) goto fail;
       tc_fence_after();
       const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
       const int si = t.si;
-      // partial output [segment][head][d] in bf16: chunk m of O holds latent
-      // columns 128 m + 64 half + (0..63) in this lane
+      // partial output [segment][head][d] in bf16: O block j holds latent
+      // columns 256 j + 128 half + (0..127) in this lane
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         uint32_t o[32];
         tmem_ld32(tl + kTmemO + c * 32, o);
         tmem_wait_ld();
-        const int d0 = 128 * (c >> 1) + 64 * half + 32 * (c & 1);
+        const int d0 = 256 * (c >> 2) + 128 * half + 32 * (c & 3);
         uint4* out = reinterpret_cast<uint4*>(part_o + ((long long)si * kH + head) * kDc + d0);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -558,7 +689,6 @@ fail:
   set_abort(sm);
 }
 
-#undef MLA_WARP_WAIT
 
 // ---------------------------------------------------------------- plan + query pack
 // The split plan (block 0) and the query packing (the other blocks) in one
@@ -598,21 +728,28 @@ __global__ void __launch_bounds__(1024) pair_plan_pack_kernel(const int32_t* __r
 }
 
 // ---------------------------------------------------------------- kernel
+template <bool kSplit>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_pair_kernel(const __grid_constant__ CUtensorMap pool, const __grid_constant__ CUtensorMap qmap,
                        const __grid_constant__ CUtensorMap qlomap, const Params p) {
+  using R = Ring<kSplit>;
   extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem<kSplit>& sm =
+      *reinterpret_cast<Smem<kSplit>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const int worker = blockIdx.x >> 1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kRing; ++s) {
-      mbar_init(&sm.full[s], 1);
+    for (int s = 0; s < kT; ++s) {
+      mbar_init(&sm.kfull[s], 1);
       mbar_init(&sm.qkd[s], 1);
       mbar_init(&sm.vfull[s], 1);
-      mbar_init(&sm.empty[s], 1);
+      mbar_init(&sm.vempty[s], 1);
+    }
+    for (int s = 0; s < R::kS; ++s) {
+      mbar_init(&sm.rfull[s], 1);
+      mbar_init(&sm.rempty[s], 1);
     }
     mbar_init(&sm.s_full, 1);
     mbar_init(&sm.s_free, 2 * kSoftmaxWarps);
@@ -623,7 +760,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(&sm.q_empty, 1);
     mbar_init(&sm.qt_full, 2 * kSoftmaxWarps);
     mbar_init(&sm.o_free, 2 * kSoftmaxWarps);
-    mbar_init(&sm.fin, 1);
+    mbar_init(&sm.fin, 2);
     mbar_init(&sm.lbar, kSoftmaxWarps);
     sm.abort_flag = 0;
     fence_mbar_init();
@@ -635,7 +772,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&pool);
     prefetch_tensormap(&qmap);
-    if (p.split) prefetch_tensormap(&qlomap);
+    if (kSplit) prefetch_tensormap(&qlomap);
   }
   tc_fence_before();
   cluster_sync();  // barriers of both CTAs initialised before any remote arrive or load
@@ -647,21 +784,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   int seg_begin = 0, seg_end = 0;
   if (worker < p.L.workers) {
     const int* wfirst = ws_at<int>(p.ws, p.L.off_worker_first);
-    seg_begin = wfirst[worker];
-    seg_end = wfirst[worker + 1];
+    seg_begin = uni(wfirst[worker]);
+    seg_end = uni(wfirst[worker + 1]);
   }
 
-  // The single-thread roles keep their warp's other lanes parked at a warp
-  // barrier (not at the CTA barrier below) while lane 0 works.
   if (warp == 0) {
-    if (lane == 0) producer_k(sm, &pool, &qmap, &qlomap, p, seg_begin, seg_end, rank);
-    __syncwarp();
+    producer_k(sm, &pool, &qmap, &qlomap, p, seg_begin, seg_end, rank, lane);
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) mma_issuer(sm, tmem, p, seg_begin, seg_end);
-    __syncwarp();
+    if (rank == 0) score_issuer(sm, tmem, p, seg_begin, seg_end, lane);
+  } else if (warp == kPvWarp) {
+    if (rank == 0) pv_issuer(sm, tmem, p, seg_begin, seg_end, lane);
   } else if (warp == kVcWarp) {
-    if (lane == 0) producer_v(sm, &pool, p, seg_begin, seg_end, rank);
-    __syncwarp();
+    producer_v(sm, &pool, p, seg_begin, seg_end, rank, lane);
   } else {
     softmax_role(sm, tmem, p, seg_begin, seg_end, rank, warp, lane);
   }
@@ -745,9 +879,11 @@ inline mla_status launch(const mla_config* c, const float* q_lat, const float* q
   if (st == MLA_OK) st = query_map(split ? qlo : qpack, rows, &qlomap);
   if (st != MLA_OK) return st;
 
-  static std::atomic<uint64_t> plan_attr{0}, plan_only_attr{0}, dec_attr{0};
+  static std::atomic<uint64_t> plan_attr{0}, plan_only_attr{0}, dec_attr{0}, dec_split_attr{0};
   const size_t plan_smem = sizeof(int) * ((size_t)rows + 1);
-  if (set_smem_once((const void*)decode_pair_kernel, kSmemBytes, dec_attr) != MLA_OK) return MLA_ERR_CUDA;
+  const void* dec_fn = split ? (const void*)decode_pair_kernel<true> : (const void*)decode_pair_kernel<false>;
+  const size_t dec_smem = split ? smem_bytes<true>() : smem_bytes<false>();
+  if (set_smem_once(dec_fn, dec_smem, split ? dec_split_attr : dec_attr) != MLA_OK) return MLA_ERR_CUDA;
   if (q_packed) {
     if (plan_smem > 48 * 1024 && set_smem_once((const void*)decode_plan_kernel, plan_smem, plan_only_attr) != MLA_OK)
       return MLA_ERR_CUDA;
@@ -763,12 +899,14 @@ inline mla_status launch(const mla_config* c, const float* q_lat, const float* q
                        k->max_blocks_per_seq, ws, L, q_lat, q_rope, rows * kH, qpack, qlo) != cudaSuccess)
       return MLA_ERR_CUDA;
   }
-  const Params p{qpack, k->block_table, seq_lens, k->max_blocks_per_seq, k->num_blocks, n_q, split ? 1 : 0,
+  const Params p{qpack,    k->block_table, seq_lens, k->max_blocks_per_seq, k->num_blocks, n_q,
                  scale * 1.4426950408889634f, wait_ns, ws, L};
-  return launch_chained(decode_pair_kernel, dim3(2 * L.workers), dim3(kThreads), kSmemBytes, s, pmap, qmap, qlomap,
-                        p) == cudaSuccess
-             ? MLA_OK
-             : MLA_ERR_CUDA;
+  const cudaError_t e =
+      split ? launch_chained(decode_pair_kernel<true>, dim3(2 * L.workers), dim3(kThreads), dec_smem, s, pmap, qmap,
+                             qlomap, p)
+            : launch_chained(decode_pair_kernel<false>, dim3(2 * L.workers), dim3(kThreads), dec_smem, s, pmap, qmap,
+                             qlomap, p);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 }  // namespace pairdec

@@ -122,12 +122,15 @@ __device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) {
   return kCluster ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity);
 }
 
+// `sleep_ns` > 0 backs off between polls (for roles that wait long while
+// other warps of the SM issue work).
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int where,
-                                          uint64_t limit_ns = kWaitLimitNs) {
+                                          uint64_t limit_ns = kWaitLimitNs, uint32_t sleep_ns = 0) {
   if (mbar_poll<kCluster>(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 0;; ++it) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_poll<kCluster>(bar, parity)) return true;
     if ((it & 255u) == 255u && global_ns() - t0 > limit_ns) {
       report(MLA_ERR_TIMEOUT, where, (int)blockIdx.x, (int)threadIdx.x);
