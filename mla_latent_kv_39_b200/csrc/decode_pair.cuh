@@ -31,9 +31,10 @@
 // the first half of the N columns and lanes 64..127 the second.
 //
 // Barriers are per tile (a ring of 4): the value-slab loads of a tile (both
-// CTAs, 8 slabs each) complete one barrier, its score MMAs commit one, its value
-// reloads complete one and its P V commits one, so the MMA thread waits and
-// commits a few times per tile and otherwise issues MMAs back to back.
+// CTAs) complete two (pairs 0-1 and 2-3), its score MMAs commit one per pair
+// (so each pair's reload starts as soon as the scores have read it), its
+// value reloads complete one and its P V commits one; the issuing threads
+// otherwise issue MMAs back to back.
 //
 // Pipeline: the score MMAs of tile i + 1 are issued as soon as the softmax
 // of tile i has copied the scores to registers (freeing them), and P V of
@@ -41,12 +42,13 @@
 // pipe interleaves the two.  Before the softmax of tile i writes P or
 // rescales O it waits for P V of tile i - 1.
 //
-// Warp roles (256 threads per CTA, each role on whole warps with one lane
-// issuing): warp 0 issues the score-side TMA loads and warp 6 the value-side
-// ones (both CTAs, counted on the leader's barriers); in the leader, warp 1
-// issues the pair's score MMAs and warp 7 its P V MMAs; warps 2..5
-// run the online softmax, one TMEM lane per thread (a head and one page of
-// the tile), and write the segment's partial output.
+// Warp roles (384 threads per CTA, each role on whole warps with one lane
+// issuing): warp 0 issues the score-side TMA loads and warp 10 the
+// value-side ones (both CTAs, counted on the leader's barriers); in the
+// leader, warp 1 issues the pair's score MMAs and warp 11 its P V MMAs;
+// warps 2..9 run the online softmax, one TMEM lane (a head and one page of
+// the tile) and 32 score columns per thread, and write the segment's
+// partial output.
 //
 // TMEM (512 columns): [0,64) the score tile, [64,320) the latent output
 // (two 128-column blocks), [320,512) the query's latent columns 0..383 (A of
@@ -90,8 +92,8 @@ constexpr int kSlab = 64 * 128;    // 64 rows x 64 bf16, 128-byte swizzle
 #define MLA_PAIR_VSLOTS_SPLIT 9
 #endif
 constexpr int kTmemS = 0, kTmemO = 64, kTmemQ = 320, kTmemCols = 512;
-constexpr int kSoftmaxWarps = 4;
-constexpr int kSoftmaxWarp0 = 2;  // warps 2..5
+constexpr int kSoftmaxWarps = 8;  // two per TMEM lane quarter, each on 32 of the tile's 64 columns
+constexpr int kSoftmaxWarp0 = 2;  // warps 2..9
 constexpr int kVcWarp = kSoftmaxWarp0 + kSoftmaxWarps;
 constexpr int kPvWarp = kVcWarp + 1;
 constexpr int kThreads = 32 * (kPvWarp + 1);
@@ -131,13 +133,15 @@ struct Smem {
   uint8_t p[2][kSlab];            // P of the tile: [page of the tile] 64 heads x 64 tokens
   uint8_t v[R::kV][2][kSlab];     // value slab pairs (score-side B, then P V B)
   uint8_t r[R::kS][kSlab];        // rotary slabs (and low query slabs)
-  uint64_t kfull[kT], qkd[kT], vfull[kT], vempty[kT];  // per tile: score loads, score MMAs, reloads, P V
+  uint64_t kfull[kT][2];  // per tile and half (pairs 0-1, 2-3): value-slab loads of both CTAs
+  uint64_t qkd[kT][kPairs];  // per tile and pair: the score MMAs have read the pair
+  uint64_t vfull[kT], vempty[kT];  // per tile: value reloads landed, P V over
   uint64_t rfull[R::kS], rempty[R::kS];                 // short ring
   uint64_t q_full, q_empty, qt_full;
   uint64_t s_full, s_free, p_full, pv_done;
-  uint64_t o_free, fin, xbar[2], lbar;
-  float xm[2][128];  // tile max of each TMEM lane (exchanged between lanes l and l ^ 64)
-  float xl[128];     // row sums at the end of a segment
+  uint64_t o_free, fin, xbar[2], lbar;  // xbar, lbar: the softmax warps' exchanges
+  float xm[2][2][128];  // [tile parity][column half] partial tile max of each TMEM lane
+  float xl[2][128];     // [column half] partial row sums at the end of a segment
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -214,9 +218,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int wh
 // warps only: the segment is read once and broadcast).
 struct Tiles {
   const int4* segs;
+  const int32_t* seq_lens;
+  int n_q;
   int si, seg_end, pg, nseg;  // nseg: segments started so far (this one included)
-  int v, pg0, pg1;            // the segment: query row, first page, end page
-  __device__ Tiles(const int4* s, int b, int e) : segs(s), si(b), seg_end(e), pg(0), nseg(1), v(0), pg0(0), pg1(0) {
+  int v, pg0, pg1, len;       // the segment: query row, first page, end page, visible rows
+  __device__ Tiles(const int4* s, const int32_t* sl, int nq, int b, int e)
+      : segs(s), seq_lens(sl), n_q(nq), si(b), seg_end(e), pg(0), nseg(1), v(0), pg0(0), pg1(0), len(0) {
     load();
     pg = pg0;
   }
@@ -226,10 +233,13 @@ struct Tiles {
       v = uni(g.x);
       pg0 = uni(g.y);
       pg1 = uni(g.z);
+      // query row v sees its sequence's rows up to and including its own
+      len = uni(seq_lens[v / n_q] - n_q + v % n_q + 1);
     }
   }
   __device__ bool valid() const { return si < seg_end; }
   __device__ int row() const { return v; }
+  __device__ int visible() const { return len; }
   __device__ bool first() const { return pg == pg0; }
   __device__ bool last() const { return pg + 2 >= pg1; }
   __device__ bool has_b() const { return pg + 1 < pg1; }
@@ -243,11 +253,6 @@ struct Tiles {
   }
 };
 
-// Visible rows of query row v: its sequence's rows up to and including its own.
-__device__ __forceinline__ int visible_len(const Params& p, int v) {
-  const int b = v / p.n_q, j = v % p.n_q;
-  return p.seq_lens[b] - p.n_q + j + 1;
-}
 
 __device__ __forceinline__ int page_valid(int len_v, int blk) { return max(0, min(kBS, len_v - blk * kBS)); }
 
@@ -277,7 +282,7 @@ __device__ void producer_k(Smem<kSplit>& sm, const CUtensorMap* pool, const CUte
   const uint64_t wns = p.wait_ns;
   int nq = 0;  // query loads issued
   int ti = 0;
-  for (Tiles t(segs, seg_begin, seg_end); t.valid() && !uni(aborted(sm) ? 1 : 0); t.next(), ++ti) {
+  for (Tiles t(segs, p.seq_lens, p.n_q, seg_begin, seg_end); t.valid() && !uni(aborted(sm) ? 1 : 0); t.next(), ++ti) {
     const int v = t.row();
     if (t.first()) {
       if (nq >= 1 && !warp_wait(&sm.q_empty, (nq - 1) & 1, 70, wns, lane)) goto fail;
@@ -291,7 +296,7 @@ __device__ void producer_k(Smem<kSplit>& sm, const CUtensorMap* pool, const CUte
     const bool has = rank == 0 || t.has_b();
     const int blk = t.pg + (int)rank;
     const int phys = has ? uni(phys_block(p, v, blk, true)) : 0;
-    const int y = has ? uni(page_valid(visible_len(p, v), blk) - kBS) : 0;
+    const int y = has ? page_valid(t.visible(), blk) - kBS : 0;
     const uint32_t page_bytes = (t.has_b() ? 2 : 1) * kSlab;
     // without split-query low slabs the short ring holds only rotary slabs: load it first
     if (!kSplit) {
@@ -301,17 +306,17 @@ __device__ void producer_k(Smem<kSplit>& sm, const CUtensorMap* pool, const CUte
       if (issue && lead) mbar_arrive_expect_tx(&sm.rfull[sl], page_bytes);
       if (issue && has) tma_load_3d_pair(sm.r[sl], pool, 64 * (kSlabs - 1), y, phys, leader(&sm.rfull[sl]));
     }
-    // the tile barrier's previous phase (tile ti - kT) is over once that tile's scores were issued
-    if (ti >= kT && !warp_wait(&sm.qkd[tslot(ti)], tpar(ti - kT), 69, wns, lane)) goto fail;
-    if (issue && lead) mbar_arrive_expect_tx(&sm.kfull[tslot(ti)], 2 * kPairs * page_bytes);
-    for (int e = 0; e < 2 * kPairs; ++e) {  // the 8 value slabs, on the tile barrier
-      const int g = ti * kPairs + (e >> 1);
+    // the tile barriers' previous phase (tile ti - kT) is over once that tile's scores were done
+    if (ti >= kT && !warp_wait(&sm.qkd[tslot(ti)][kPairs - 1], tpar(ti - kT), 69, wns, lane)) goto fail;
+    for (int e = 0; e < 2 * kPairs; ++e) {  // the 8 value slabs, on the tile's half barriers
+      const int g = ti * kPairs + (e >> 1), h = e >> 2;
       if ((e & 1) == 0 && g >= R::kV) {  // the double slot's previous tile is past its P V
         const int tp = (g - R::kV) / kPairs;
         if (!warp_wait(&sm.vempty[tslot(tp)], tpar(tp), 71, wns, lane)) goto fail;
       }
+      if (issue && lead && (e & 3) == 0) mbar_arrive_expect_tx(&sm.kfull[tslot(ti)][h], 4 * page_bytes);
       if (issue && has)
-        tma_load_3d_pair(sm.v[g % R::kV][e & 1], pool, 64 * e, y, phys, leader(&sm.kfull[tslot(ti)]));
+        tma_load_3d_pair(sm.v[g % R::kV][e & 1], pool, 64 * e, y, phys, leader(&sm.kfull[tslot(ti)][h]));
     }
     // then (split-query mode) the short-ring items in their order (the score MMAs free them one by one)
     for (int k = 0; kSplit && k < R::kPerTile; ++k) {
@@ -345,22 +350,22 @@ __device__ void producer_v(Smem<kSplit>& sm, const CUtensorMap* pool, const Para
   const int4* segs = ws_at<int4>(p.ws, p.L.off_seg);
   const bool lead = rank == 0, issue = lane == 0;
   int ti = 0;
-  for (Tiles t(segs, seg_begin, seg_end); t.valid() && !uni(aborted(sm) ? 1 : 0); t.next(), ++ti) {
-    const int v = t.row(), len_v = uni(visible_len(p, v));
-    if (!warp_wait(&sm.qkd[tslot(ti)], tpar(ti), 73, p.wait_ns, lane)) goto fail;
+  for (Tiles t(segs, p.seq_lens, p.n_q, seg_begin, seg_end); t.valid() && !uni(aborted(sm) ? 1 : 0); t.next(), ++ti) {
+    const int v = t.row(), len_v = t.visible();
     // pairs 0 and 2 read page 0, pairs 1 and 3 page 1 (absent in a one-page tile)
     if (issue && lead) mbar_arrive_expect_tx(&sm.vfull[tslot(ti)], (t.has_b() ? 4 : 2) * 2 * kSlab);
-    // this CTA reloads the pairs m with m mod 2 != rank, all from page 1 - rank
+    // this CTA reloads the pairs m with m mod 2 != rank, all from page 1 - rank,
+    // each once the scores have read it
     const int pgi = 1 - (int)rank;
-    if (pgi == 0 || t.has_b()) {
-      const int blk = t.pg + pgi;
-      const int y = page_valid(len_v, blk) - kBS, phys = uni(phys_block(p, v, blk, false));
-      for (int m = pgi; m < kPairs; m += 2) {
-        const int ds = R::vslot(ti, m), x = 128 * (m ^ 1);
-        if (issue) {
-          tma_load_3d_pair(sm.v[ds][0], pool, x, y, phys, leader(&sm.vfull[tslot(ti)]));
-          tma_load_3d_pair(sm.v[ds][1], pool, x + 64, y, phys, leader(&sm.vfull[tslot(ti)]));
-        }
+    const bool exists = pgi == 0 || t.has_b();
+    const int blk = t.pg + pgi;
+    const int y = exists ? page_valid(len_v, blk) - kBS : 0, phys = exists ? uni(phys_block(p, v, blk, false)) : 0;
+    for (int m = pgi; m < kPairs; m += 2) {
+      if (!warp_wait(&sm.qkd[tslot(ti)][m], tpar(ti), 73, p.wait_ns, lane)) goto fail;
+      const int ds = R::vslot(ti, m), x = 128 * (m ^ 1);
+      if (issue && exists) {
+        tma_load_3d_pair(sm.v[ds][0], pool, x, y, phys, leader(&sm.vfull[tslot(ti)]));
+        tma_load_3d_pair(sm.v[ds][1], pool, x + 64, y, phys, leader(&sm.vfull[tslot(ti)]));
       }
     }
   }
@@ -393,10 +398,12 @@ __device__ bool issue_scores(Smem<kSplit>& sm, uint32_t tmem, const Tiles& t, in
                     !warp_wait(&sm.qt_full, (t.nseg - 1) & 1, 79, wns, lane)))
     return false;
   if (ti >= 1 && !warp_wait(&sm.s_free, (ti - 1) & 1, 81, wns, lane)) return false;
-  if (!warp_wait(&sm.kfull[tslot(ti)], tpar(ti), 82, wns, lane)) return false;
-  tc_fence_after();
 #pragma unroll
   for (int e = 0; e < kSlabs; ++e) {
+    if (e == 0 || e == 4) {
+      if (!warp_wait(&sm.kfull[tslot(ti)][e >> 2], tpar(ti), 82, wns, lane)) return false;
+      tc_fence_after();
+    }
     if (e == kSlabs - 1) {
       if (!warp_wait(&sm.rfull[rope_sl], R::suse(ti, R::kRope) & 1, 78, wns, lane)) return false;
       tc_fence_after();
@@ -426,9 +433,9 @@ __device__ bool issue_scores(Smem<kSplit>& sm, uint32_t tmem, const Tiles& t, in
         mma_commit_pair(&sm.rempty[lo_sl], kBoth);
       }
     }
+    if (issue && (e & 1) && e < 2 * kPairs) mma_commit_pair(&sm.qkd[tslot(ti)][e >> 1], kBoth);
   }
   if (issue) {
-    mma_commit_pair(&sm.qkd[tslot(ti)], kBoth);
     mma_commit_pair(&sm.rempty[rope_sl], kBoth);
     mma_commit_pair(&sm.s_full, kBoth);
     if (t.last()) mma_commit_pair(&sm.q_empty, kBoth);
@@ -486,7 +493,7 @@ __device__ void score_issuer(Smem<kSplit>& sm, uint32_t tmem, const Params& p, i
   const uint64_t wns = p.wait_ns;
   int ti = 0;
   bool ok = true;
-  for (Tiles t(segs, seg_begin, seg_end); t.valid() && ok; t.next(), ++ti) ok = issue_scores(sm, tmem, t, ti, wns, lane);
+  for (Tiles t(segs, p.seq_lens, p.n_q, seg_begin, seg_end); t.valid() && ok; t.next(), ++ti) ok = issue_scores(sm, tmem, t, ti, wns, lane);
   if (!ok) set_abort(sm);
   if (lane == 0) mma_commit_pair(&sm.fin, 1);
   warp_wait(&sm.fin, 0, 87, wns, lane);
@@ -498,7 +505,7 @@ __device__ void pv_issuer(Smem<kSplit>& sm, uint32_t tmem, const Params& p, int 
   const uint64_t wns = p.wait_ns;
   int ti = 0;
   bool ok = true;
-  for (Tiles t(segs, seg_begin, seg_end); t.valid() && ok; t.next(), ++ti) ok = issue_pv(sm, tmem, t, ti, wns, lane);
+  for (Tiles t(segs, p.seq_lens, p.n_q, seg_begin, seg_end); t.valid() && ok; t.next(), ++ti) ok = issue_pv(sm, tmem, t, ti, wns, lane);
   if (!ok) set_abort(sm);
   if (lane == 0) mma_commit_pair(&sm.fin, 1);
   warp_wait(&sm.fin, 0, 88, wns, lane);
@@ -507,25 +514,28 @@ __device__ void pv_issuer(Smem<kSplit>& sm, uint32_t tmem, const Params& p, int 
 // ---------------------------------------------------------------- softmax
 
 // The query's latent columns 0..383 of this lane's head into TMEM (the A
-// operand of the first 24 score K steps).  A pair MMA with A in TMEM reads
-// each CTA's 64 rows from lanes 0..63 and again from lanes 64..127, so lanes
-// l and l ^ 64 both hold head 64 r + (l mod 64).  Then the leader is told.
+// operand of the first 24 score K steps); the two warps of a lane quarter
+// take 192 columns each.  A pair MMA with A in TMEM reads each CTA's 64 rows
+// from lanes 0..63 and again from lanes 64..127, so lanes l and l ^ 64 both
+// hold head 64 r + (l mod 64).  Then the leader is told.
 template <bool kSplit>
 __device__ __forceinline__ void load_query_tmem(Smem<kSplit>& sm, const Params& p, int v, int head, uint32_t tl,
-                                                int lane) {
-  const uint4* src = reinterpret_cast<const uint4*>(p.q + ((long long)v * kH + head) * kRow);
+                                                int ch, int lane) {
+  constexpr int kCols = kTmemQSlabs * 32 / 2;  // TMEM columns per warp (bf16 pairs): 96
+  static_assert(kCols % 32 == 0, "query columns per warp in rounds of 32");
+  const uint4* src = reinterpret_cast<const uint4*>(p.q + ((long long)v * kH + head) * kRow) + ch * (kCols / 4);
 #pragma unroll 1
-  for (int b = 0; b < kTmemQSlabs / 2; ++b) {  // 16 loads in flight per round, 64 columns each
-    uint4 w[16];
+  for (int b = 0; b < kCols / 32; ++b) {  // 8 loads in flight per round, 32 columns each
+    uint4 w[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) w[i] = __ldg(src + b * 16 + i);
+    for (int i = 0; i < 8; ++i) w[i] = __ldg(src + b * 8 + i);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       const uint32_t x[16] = {w[4 * c].x,     w[4 * c].y,     w[4 * c].z,     w[4 * c].w,
                               w[4 * c + 1].x, w[4 * c + 1].y, w[4 * c + 1].z, w[4 * c + 1].w,
                               w[4 * c + 2].x, w[4 * c + 2].y, w[4 * c + 2].z, w[4 * c + 2].w,
                               w[4 * c + 3].x, w[4 * c + 3].y, w[4 * c + 3].z, w[4 * c + 3].w};
-      tmem_st16(tl + kTmemQ + b * 64 + c * 16, x);
+      tmem_st16(tl + kTmemQ + ch * kCols + b * 32 + c * 16, x);
     }
   }
   tmem_wait_st();
@@ -534,11 +544,18 @@ __device__ __forceinline__ void load_query_tmem(Smem<kSplit>& sm, const Params& 
   if (lane == 0) mbar_arrive_remote(leader(&sm.qt_full));
 }
 
+// Online softmax, one TMEM lane (a head and a page of the tile) and 32 of
+// its 64 score columns per thread: warp w handles lane quarter w mod 4 and
+// column half ch.  The row max and (at the end of a segment) the row sum of
+// a head combine the four threads of its two lanes and two halves through
+// shared memory and an mbarrier of the softmax warps (a bounded wait).
+
 template <bool kSplit>
 __device__ void softmax_role(Smem<kSplit>& sm, uint32_t tmem, const Params& p, int seg_begin, int seg_end,
                              uint32_t rank, int warp, int lane) {
   const int4* segs = ws_at<int4>(p.ws, p.L.off_seg);
   const int qw = warp & 3;                                 // TMEM lane quarter
+  const int ch = (warp - kSoftmaxWarp0) >> 2;              // column half of the tile / of O
   const int l = qw * 32 + lane;                            // TMEM lane
   const int half = l >> 6;                                 // page of the tile / column half of each O block
   const int hl = l & 63, head = kHalfH * (int)rank + hl;   // head of this lane
@@ -549,51 +566,46 @@ __device__ void softmax_role(Smem<kSplit>& sm, uint32_t tmem, const Params& p, i
 
   float m_used = -INFINITY, lsum = 0.f;
   int nseg_done = 0;
-  Tiles t(segs, seg_begin, seg_end);
-  if (t.valid()) load_query_tmem(sm, p, t.row(), head, tl, lane);
+  Tiles t(segs, p.seq_lens, p.n_q, seg_begin, seg_end);
+  if (t.valid()) load_query_tmem(sm, p, t.row(), head, tl, ch, lane);
   for (int i = 0; t.valid(); ++i, t.next()) {
-    const int v = t.row(), len_v = visible_len(p, v);
     const bool first = t.first(), last = t.last();
     if (first) {
       m_used = -INFINITY;
       lsum = 0.f;
     }
+    // this lane's page: rows past the visible length sit at the top of the tile
+    const int shift = kBS - ((half == 0 || t.has_b()) ? page_valid(t.visible(), t.pg + half) : 0) - 32 * ch;
     if (!warp_wait(&sm.s_full, i & 1, 90, wns, lane, MLA_SOFTMAX_SLEEP_NS)) goto fail;
     tc_fence_after();
-    float s[64];
+    float s[32];
     {
-      uint32_t a[32], b[32];
-      tmem_ld32(tl + kTmemS, a);
-      tmem_ld32(tl + kTmemS + 32, b);
+      uint32_t a[32];
+      tmem_ld32(tl + kTmemS + 32 * ch, a);
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        s[c] = __uint_as_float(a[c]);
-        s[32 + c] = __uint_as_float(b[c]);
-      }
+      for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(a[c]);
     }
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive_remote(leader(&sm.s_free));
 
-    // this lane's page: rows past the visible length sit at the top of the tile
-    const int blk = t.pg + half;
-    const int shift = kBS - ((half == 0 || t.has_b()) ? page_valid(len_v, blk) : 0);
     float m8[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) m8[c] = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < 64; ++c) {
+    for (int c = 0; c < 32; ++c) {
       s[c] = c >= shift ? s[c] * p.scale_log2 : -INFINITY;
       m8[c & 7] = fmaxf(m8[c & 7], s[c]);
     }
     const float m_loc =
         fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-    sm.xm[i & 1][l] = m_loc;
+    sm.xm[i & 1][ch][l] = m_loc;
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.xbar[i & 1]);
     if (!warp_wait(&sm.xbar[i & 1], (i >> 1) & 1, 91, wns, lane)) goto fail;
-    const float m_tile = fmaxf(m_loc, sm.xm[i & 1][l ^ 64]);
+    const float m_tile = fmaxf(fmaxf(sm.xm[i & 1][0][l], sm.xm[i & 1][1][l]),
+                               fmaxf(sm.xm[i & 1][0][l ^ 64], sm.xm[i & 1][1][l ^ 64]));
 
     bool rescale = false;
     float alpha = 1.f;
@@ -605,10 +617,10 @@ __device__ void softmax_role(Smem<kSplit>& sm, uint32_t tmem, const Params& p, i
       rescale = true;
     }
     const float mbase = m_used == -INFINITY ? 0.f : m_used;
-    uint32_t pk[32];
+    uint32_t pk[16];
     float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
+    for (int c = 0; c < 16; ++c) {
       const float p0 = fast_exp2(s[2 * c] - mbase), p1 = fast_exp2(s[2 * c + 1] - mbase);
       ps[c & 3] += p0 + p1;
       pk[c] = pack_bf16x2(p0, p1);
@@ -619,10 +631,11 @@ __device__ void softmax_role(Smem<kSplit>& sm, uint32_t tmem, const Params& p, i
     // over before this tile rescales O or overwrites P.
     if (i >= 1 && !warp_wait(&sm.pv_done, (i - 1) & 1, 92, wns, lane)) goto fail;
     tc_fence_after();
-    // tcgen05.ld / st are warp-collective: the warp rescales when any lane needs it.
+    // tcgen05.ld / st are warp-collective: the warp rescales (its 4 of the
+    // lane's 8 O chunks) when any lane needs it.
     if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 4 * ch; c < 4 * ch + 4; ++c) {
         uint32_t o[32];
         const uint32_t a = tl + kTmemO + c * 32;
         tmem_ld32(a, o);
@@ -634,11 +647,12 @@ __device__ void softmax_role(Smem<kSplit>& sm, uint32_t tmem, const Params& p, i
       tmem_wait_st();
     }
     {
-      // row hl of this page's P slab, K-major with the 128-byte swizzle
+      // row hl of this page's P slab, K-major with the 128-byte swizzle:
+      // 16-byte chunks 4 ch .. 4 ch + 3
       uint8_t* row = sm.p[half] + hl * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(row + ((c ^ (hl & 7)) << 4)) =
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(row + (((4 * ch + c) ^ (hl & 7)) << 4)) =
             make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
     }
     fence_proxy_async_smem();
@@ -648,23 +662,24 @@ __device__ void softmax_role(Smem<kSplit>& sm, uint32_t tmem, const Params& p, i
 
     // The scores of this segment are all done (s_full of its last tile): the
     // next segment's query can replace this one in TMEM before the epilogue.
-    if (last && t.si + 1 < seg_end) load_query_tmem(sm, p, segs[t.si + 1].x, head, tl, lane);
+    if (last && t.si + 1 < seg_end) load_query_tmem(sm, p, segs[t.si + 1].x, head, tl, ch, lane);
 
     if (last) {
       // epilogue of the segment: O / l and the log2-sum-exp
-      sm.xl[l] = lsum;
+      sm.xl[ch][l] = lsum;
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.lbar);
       if (!warp_wait(&sm.lbar, nseg_done & 1, 94, wns, lane)) goto fail;
-      const float ltot = lsum + sm.xl[l ^ 64];
+      const float ltot = (sm.xl[0][l] + sm.xl[1][l]) + (sm.xl[0][l ^ 64] + sm.xl[1][l ^ 64]);
       if (!warp_wait(&sm.pv_done, i & 1, 95, wns, lane)) goto fail;
       tc_fence_after();
       const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
       const int si = t.si;
       // partial output [segment][head][d] in bf16: O block j holds latent
-      // columns 256 j + 128 half + (0..127) in this lane
+      // columns 256 j + 128 half + (0..127) in this lane; this warp writes
+      // block ch
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 4 * ch; c < 4 * ch + 4; ++c) {
         uint32_t o[32];
         tmem_ld32(tl + kTmemO + c * 32, o);
         tmem_wait_ld();
@@ -677,7 +692,7 @@ __device__ void softmax_role(Smem<kSplit>& sm, uint32_t tmem, const Params& p, i
                               pack_bf16x2(f[4] * inv, f[5] * inv), pack_bf16x2(f[6] * inv, f[7] * inv));
         }
       }
-      if (half == 0) part_lse[(long long)si * kH + head] = ltot > 0.f ? m_used + log2f(ltot) : -INFINITY;
+      if (half == 0 && ch == 0) part_lse[(long long)si * kH + head] = ltot > 0.f ? m_used + log2f(ltot) : -INFINITY;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(leader(&sm.o_free));
@@ -688,7 +703,6 @@ __device__ void softmax_role(Smem<kSplit>& sm, uint32_t tmem, const Params& p, i
 fail:
   set_abort(sm);
 }
-
 
 // ---------------------------------------------------------------- plan + query pack
 // The split plan (block 0) and the query packing (the other blocks) in one
@@ -742,8 +756,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kT; ++s) {
-      mbar_init(&sm.kfull[s], 1);
-      mbar_init(&sm.qkd[s], 1);
+      for (int h = 0; h < 2; ++h) mbar_init(&sm.kfull[s][h], 1);
+      for (int m = 0; m < kPairs; ++m) mbar_init(&sm.qkd[s][m], 1);
       mbar_init(&sm.vfull[s], 1);
       mbar_init(&sm.vempty[s], 1);
     }
@@ -755,13 +769,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(&sm.s_free, 2 * kSoftmaxWarps);
     mbar_init(&sm.p_full, 2 * kSoftmaxWarps);
     mbar_init(&sm.pv_done, 1);
-    for (int b = 0; b < 2; ++b) mbar_init(&sm.xbar[b], kSoftmaxWarps);
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
     mbar_init(&sm.qt_full, 2 * kSoftmaxWarps);
     mbar_init(&sm.o_free, 2 * kSoftmaxWarps);
-    mbar_init(&sm.fin, 2);
+    for (int b = 0; b < 2; ++b) mbar_init(&sm.xbar[b], kSoftmaxWarps);
     mbar_init(&sm.lbar, kSoftmaxWarps);
+    mbar_init(&sm.fin, 2);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
