@@ -296,10 +296,10 @@ def run_ours(args):
     def one_step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        layer.append_and_queries(x, seq_idx, pos)
+        layer.append_and_queries(x, seq_idx, pos, seq_lens=seq_lens)   # the split plan beside the projections
         if ev is not None:
             ev[1].record(stream)
-        layer.decode(seq_lens)
+        layer.decode(seq_lens, planned=layer.packed)
         if ev is not None:
             ev[2].record(stream)
         if not layer.fused_out:     # bf16: the split merge runs inside the W_UV projection
@@ -397,7 +397,7 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                      "traffic": traffic,
-                     "kernel": "mla_decode call (plan, query pack and decode kernels)",
+                     "kernel": "mla_decode_packed_planned call (the pair decode kernel; its split plan runs beside the query projections)",
                      "algorithmic_bytes_per_launch": cache_bytes,
                      "peak_source": peaks["source"]},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,

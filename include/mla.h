@@ -240,6 +240,30 @@ mla_status mla_decode_packed(const mla_config* cfg, const void* q_packed, int32_
                              void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * The decode's split plan on its own (not on the pages: how the cached pages
+ * are cut among the SMs).  The plan depends only on seq_lens, the cache's
+ * block geometry, batch, n_q and max_workers, so a caller can compute it
+ * early (e.g. on a second stream beside the query projections) and then run
+ * mla_decode_packed_planned, which skips it.
+ *   mla_decode_plan: writes the plan into `workspace` (the region
+ *     mla_decode_packed would write); arguments as in mla_decode_packed.
+ *   mla_decode_packed_planned: mla_decode_packed without the planning launch;
+ *     `workspace` must hold the plan of an mla_decode_plan call with the same
+ *     cfg, batch, n_q, cache geometry, seq_lens contents and max_workers,
+ *     ordered before this call (same stream, or an event).  Results are
+ *     identical to mla_decode_packed.  A plan that does not match these
+ *     arguments is caught only partly (its header is checked by the decode and
+ *     the merge; a stale plan for other sequence lengths gives wrong output).
+ * Errors as mla_decode_packed.
+ * ------------------------------------------------------------------------- */
+mla_status mla_decode_plan(const mla_config* cfg, int32_t batch, int32_t n_q, const mla_cache* cache,
+                           const int32_t* seq_lens, int32_t max_workers, void* workspace, size_t ws_bytes,
+                           void* stream);
+mla_status mla_decode_packed_planned(const mla_config* cfg, const void* q_packed, int32_t batch, int32_t n_q,
+                                     const mla_cache* cache, const int32_t* seq_lens, int32_t max_workers,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Step 4a - split combine (not on the pages; the standard log-sum-exp merge):
  *   o_lat[t,h] = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),  M = max_s lse_s
  * over the partials that mla_decode left in `workspace` (same batch, n_q).

@@ -22,6 +22,8 @@ from .abi import (  # noqa: F401
     mla_combine_out_proj_workspace_size,
     mla_decode,
     mla_decode_packed,
+    mla_decode_packed_planned,
+    mla_decode_plan,
     mla_decode_workspace_size,
     mla_get_device_error,
     mla_kernel_launches,

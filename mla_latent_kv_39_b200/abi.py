@@ -66,6 +66,8 @@ SIGNATURES = {
     "mla_query_packed_bytes": (_sz, [_P_CFG, _i32]),
     "mla_absorb_q_packed": (_i32, [_P_CFG, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mla_decode_packed": (_i32, [_P_CFG, _vp, _i32, _i32, _P_CACHE, _vp, _i32, _vp, _sz, _vp]),
+    "mla_decode_packed_planned": (_i32, [_P_CFG, _vp, _i32, _i32, _P_CACHE, _vp, _i32, _vp, _sz, _vp]),
+    "mla_decode_plan": (_i32, [_P_CFG, _i32, _i32, _P_CACHE, _vp, _i32, _vp, _sz, _vp]),
     "mla_decode_workspace_size": (_sz, [_P_CFG, _i32, _i32, _i32]),
     "mla_decode": (_i32, [_P_CFG, _vp, _vp, _i32, _i32, _P_CACHE, _vp, _i32, _vp, _sz, _vp]),
     "mla_combine": (_i32, [_P_CFG, _vp, _sz, _i32, _i32, _vp, _vp]),
@@ -295,6 +297,27 @@ def mla_decode_packed(cfg: Config, q_packed, batch: int, n_q: int, cache: Cache,
     _check(lib().mla_decode_packed(ctypes.byref(cfg.c()), _ptr(q_packed), batch, n_q, ctypes.byref(cache.c),
                                    _ptr(seq_lens), max_workers, _ptr(workspace), workspace.numel(),
                                    _stream(stream)), "mla_decode_packed")
+
+
+def mla_decode_plan(cfg: Config, batch: int, n_q: int, cache: Cache, seq_lens, workspace, max_workers: int = 0,
+                    stream=None):
+    _need(seq_lens, "seq_lens", torch.int32, shape=(batch,))
+    _need(workspace, "workspace", torch.uint8)
+    _check(lib().mla_decode_plan(ctypes.byref(cfg.c()), batch, n_q, ctypes.byref(cache.c), _ptr(seq_lens),
+                                 max_workers, _ptr(workspace), workspace.numel(), _stream(stream)),
+           "mla_decode_plan")
+
+
+def mla_decode_packed_planned(cfg: Config, q_packed, batch: int, n_q: int, cache: Cache, seq_lens, workspace,
+                              max_workers: int = 0, stream=None):
+    H = cfg.n_heads
+    _need(q_packed, "q_packed", torch.bfloat16,
+          shape=((2 if cfg.split_query else 1) * batch * n_q, H, cfg.d_c + cfg.d_r))
+    _need(seq_lens, "seq_lens", torch.int32, shape=(batch,))
+    _need(workspace, "workspace", torch.uint8)
+    _check(lib().mla_decode_packed_planned(ctypes.byref(cfg.c()), _ptr(q_packed), batch, n_q,
+                                           ctypes.byref(cache.c), _ptr(seq_lens), max_workers, _ptr(workspace),
+                                           workspace.numel(), _stream(stream)), "mla_decode_packed_planned")
 
 
 def mla_decode(cfg: Config, q_lat, q_rope, batch: int, n_q: int, cache: Cache, seq_lens, workspace,

@@ -882,7 +882,7 @@ inline mla_status set_smem_once(const void* fn, size_t bytes, std::atomic<uint64
 // mla_absorb_q_packed) the first launch only computes the plan.
 inline mla_status launch(const mla_config* c, const float* q_lat, const float* q_rope, const bf16* q_packed, int n_q,
                          const mla_cache* k, const int32_t* seq_lens, void* ws, const DecodeLayout& L, float scale,
-                         unsigned long long wait_ns, cudaStream_t s) {
+                         unsigned long long wait_ns, cudaStream_t s, bool planned = false) {
   const bool split = (c->flags & MLA_FLAG_SPLIT_QUERY) != 0;
   const long long rows = (long long)L.batch * L.n_q;
   bf16* qpack = q_packed ? const_cast<bf16*>(q_packed) : reinterpret_cast<bf16*>(static_cast<char*>(ws) + L.off_qpack);
@@ -899,11 +899,14 @@ inline mla_status launch(const mla_config* c, const float* q_lat, const float* q
   const size_t dec_smem = split ? smem_bytes<true>() : smem_bytes<false>();
   if (set_smem_once(dec_fn, dec_smem, split ? dec_split_attr : dec_attr) != MLA_OK) return MLA_ERR_CUDA;
   if (q_packed) {
-    if (plan_smem > 48 * 1024 && set_smem_once((const void*)decode_plan_kernel, plan_smem, plan_only_attr) != MLA_OK)
-      return MLA_ERR_CUDA;
-    if (launch_chained(decode_plan_kernel, dim3(1), dim3(1024), plan_smem, s, seq_lens, c->block_size,
-                       k->max_blocks_per_seq, ws, L) != cudaSuccess)
-      return MLA_ERR_CUDA;
+    if (!planned) {
+      if (plan_smem > 48 * 1024 &&
+          set_smem_once((const void*)decode_plan_kernel, plan_smem, plan_only_attr) != MLA_OK)
+        return MLA_ERR_CUDA;
+      if (launch_chained(decode_plan_kernel, dim3(1), dim3(1024), plan_smem, s, seq_lens, c->block_size,
+                         k->max_blocks_per_seq, ws, L) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    }
   } else {
     if (plan_smem > 48 * 1024 && set_smem_once((const void*)pair_plan_pack_kernel, plan_smem, plan_attr) != MLA_OK)
       return MLA_ERR_CUDA;

@@ -511,9 +511,9 @@ mla_status mla_absorb_q_packed(const mla_config* cfg, const void* x, int32_t n_t
                    static_cast<cudaStream_t>(stream));
 }
 
-mla_status mla_decode_packed(const mla_config* cfg, const void* q_packed, int32_t batch, int32_t n_q,
-                             const mla_cache* cache, const int32_t* seq_lens, int32_t max_workers, void* workspace,
-                             size_t ws_bytes, void* stream) {
+static mla_status decode_packed_impl(const mla_config* cfg, const void* q_packed, int32_t batch, int32_t n_q,
+                                     const mla_cache* cache, const int32_t* seq_lens, int32_t max_workers,
+                                     void* workspace, size_t ws_bytes, void* stream, bool planned) {
   MLA_TRY(check_cfg(cfg));
   if (batch < 0 || n_q <= 0 || max_workers < 0) return MLA_ERR_INVALID_ARG;
   if (batch == 0) return MLA_OK;
@@ -528,7 +528,44 @@ mla_status mla_decode_packed(const mla_config* cfg, const void* q_packed, int32_
   if (ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
   return pairdec::launch(cfg, nullptr, nullptr, static_cast<const bf16*>(q_packed), n_q, cache, seq_lens, workspace,
                          L, scale_of(cfg), g_wait_limit_ns.load(std::memory_order_relaxed),
-                         static_cast<cudaStream_t>(stream));
+                         static_cast<cudaStream_t>(stream), planned);
+}
+
+mla_status mla_decode_packed(const mla_config* cfg, const void* q_packed, int32_t batch, int32_t n_q,
+                             const mla_cache* cache, const int32_t* seq_lens, int32_t max_workers, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  return decode_packed_impl(cfg, q_packed, batch, n_q, cache, seq_lens, max_workers, workspace, ws_bytes, stream,
+                            false);
+}
+
+mla_status mla_decode_packed_planned(const mla_config* cfg, const void* q_packed, int32_t batch, int32_t n_q,
+                                     const mla_cache* cache, const int32_t* seq_lens, int32_t max_workers,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  return decode_packed_impl(cfg, q_packed, batch, n_q, cache, seq_lens, max_workers, workspace, ws_bytes, stream,
+                            true);
+}
+
+mla_status mla_decode_plan(const mla_config* cfg, int32_t batch, int32_t n_q, const mla_cache* cache,
+                           const int32_t* seq_lens, int32_t max_workers, void* workspace, size_t ws_bytes,
+                           void* stream) {
+  MLA_TRY(check_cfg(cfg));
+  if (batch < 0 || n_q <= 0 || max_workers < 0) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!seq_lens || !workspace) return MLA_ERR_INVALID_ARG;
+  if ((long long)batch * n_q > kPlanMaxRows) return MLA_ERR_UNSUPPORTED;
+  MLA_TRY(check_cache(cache));
+  if (cache->batch < batch) return MLA_ERR_INVALID_ARG;
+  if (!all_aligned16(workspace)) return MLA_ERR_INVALID_ARG;
+  const DecodeLayout L = decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers),
+                                       qpack_row_bytes(cfg), part_elem(cfg));
+  if (ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
+  const size_t plan_smem = sizeof(int) * ((size_t)batch * n_q + 1);
+  static std::atomic<uint64_t> attr{0};
+  if (plan_smem > 48 * 1024 && pairdec::set_smem_once((const void*)decode_plan_kernel, plan_smem, attr) != MLA_OK)
+    return MLA_ERR_CUDA;
+  MLA_CUDA(launch_chained(decode_plan_kernel, dim3(1), dim3(1024), plan_smem, static_cast<cudaStream_t>(stream),
+                          seq_lens, cfg->block_size, cache->max_blocks_per_seq, workspace, L));
+  return MLA_OK;
 }
 
 size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t n_q, int32_t max_workers) {

@@ -84,10 +84,12 @@ class DecodeLayer:
             q = q + self.q_packed[n:].float()
         return q[..., :self.cfg.d_c], q[..., self.cfg.d_c:]
 
-    def append_and_queries(self, x, seq_idx, pos, stream=None):
+    def append_and_queries(self, x, seq_idx, pos, stream=None, seq_lens=None):
         """The append and the query projections of one step, overlapped: the
         projections go first on ``stream`` (so their CTAs are placed first), the
-        append on a side stream; ``stream`` waits for both before returning."""
+        append on a side stream; ``stream`` waits for both before returning.
+        With ``seq_lens`` (packed-query path) the side stream also computes the
+        decode's split plan, and the next ``decode(..., planned=True)`` skips it."""
         main = stream or torch.cuda.current_stream()
         ready = torch.cuda.Event()
         ready.record(main)
@@ -98,15 +100,25 @@ class DecodeLayer:
             self.ws_append = torch.empty(need, dtype=torch.uint8, device=self.ws_append.device)
         abi.mla_cache_append(self.cfg, x, self.W["W_DKV"], self.W["W_KR"], seq_idx, pos, self.cache,
                              self.ws_append, self.side)
+        keep = [x, seq_idx, pos]
+        if seq_lens is not None and self.packed:
+            abi.mla_decode_plan(self.cfg, self.batch, self.n_q, self.cache, seq_lens, self.ws_decode,
+                                self.max_workers, self.side)
+            keep.append(seq_lens)
         done = torch.cuda.Event()
         done.record(self.side)
         main.wait_event(done)
         # keep the inputs alive until the side stream has used them
-        for t in (x, seq_idx, pos):
+        for t in keep:
             t.record_stream(self.side)
 
-    def decode(self, seq_lens, stream=None):
-        if self.packed:
+    def decode(self, seq_lens, stream=None, planned=False):
+        """Split-KV decode; ``planned``: the plan is already in the workspace
+        (``append_and_queries`` with ``seq_lens``, same sequence lengths)."""
+        if self.packed and planned:
+            abi.mla_decode_packed_planned(self.cfg, self.q_packed, self.batch, self.n_q, self.cache, seq_lens,
+                                          self.ws_decode, self.max_workers, stream)
+        elif self.packed:
             abi.mla_decode_packed(self.cfg, self.q_packed, self.batch, self.n_q, self.cache, seq_lens,
                                   self.ws_decode, self.max_workers, stream)
         else:
@@ -135,8 +147,8 @@ class DecodeLayer:
     def step(self, x, seq_idx, pos, seq_lens, stream=None, want_o_lat: bool = False) -> torch.Tensor:
         """Device-resident step: returns ``y`` ``[batch * n_q, hidden]`` (a reused buffer).
         ``want_o_lat`` also fills ``self.o_lat`` (always filled on the fp32 path)."""
-        self.append_and_queries(x, seq_idx, pos, stream)
-        self.decode(seq_lens, stream)
+        self.append_and_queries(x, seq_idx, pos, stream, seq_lens=seq_lens)
+        self.decode(seq_lens, stream, planned=self.packed)
         if want_o_lat or not self.fused_out:
             self.combine(stream)
         self.project(stream)
@@ -187,8 +199,8 @@ class DecodeLayer:
             if between is not None:
                 between(k)
             x, seq_idx, pos, seq_lens = dbuf[k % 2]
-            self.append_and_queries(x, seq_idx, pos, stream)
-            self.decode(seq_lens, stream)
+            self.append_and_queries(x, seq_idx, pos, stream, seq_lens=seq_lens)
+            self.decode(seq_lens, stream, planned=self.packed)
             if not self.fused_out:
                 self.combine(stream)
             self.project(stream, y=ybuf[k % 2])

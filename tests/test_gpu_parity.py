@@ -228,3 +228,20 @@ def test_fp32_query_handoff_gives_the_packed_paths_result():
     assert torch.equal(a.o_lat, b.o_lat)
     assert torch.equal(a.y, b.y)
 
+
+
+def test_plan_on_the_side_stream_gives_the_same_result():
+    """step() computes the split plan with mla_decode_plan beside the query
+    projections and decodes with mla_decode_packed_planned; planning inside
+    mla_decode_packed gives identical o_lat and y."""
+    wl = reduced(WORKLOADS["v3_b64_ragged1k_8k"], lengths=[3000, 70, 1500, 1])
+    data, dev, layer = run_gpu(wl, max_workers=9)
+    o_a, y_a = layer.o_lat.clone(), layer.y.clone()
+    layer.ws_decode.zero_()
+    layer.decode(dev["seq_lens"])                 # plan + decode in one call
+    layer.combine()
+    layer.project()
+    torch.cuda.synchronize()
+    check_device_error()
+    assert torch.equal(layer.o_lat, o_a)
+    assert torch.equal(layer.y, y_a)
