@@ -304,6 +304,9 @@ mla_status mla_out_proj(const mla_config* cfg, const float* o_lat, int32_t n_tok
  *   workspace >= mla_combine_out_proj_workspace_size(cfg, batch, n_q) bytes
  * bf16 storage only (MLA_ERR_UNSUPPORTED otherwise, or when v_head != 128 or
  * the decode has more than 512 segments: batch n_q + workers - 1 > 512).
+ * mla_combine_out_proj_workspace_size returns 0 for shapes the fused path
+ * does not take at the default worker count (then use mla_combine +
+ * mla_out_proj).
  * A decode workspace that mla_decode did not write for this batch makes y
  * zero and records MLA_ERR_WORKSPACE on the device error word.
  * ------------------------------------------------------------------------- */

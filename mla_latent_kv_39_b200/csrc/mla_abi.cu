@@ -624,6 +624,11 @@ mla_status mla_combine(const mla_config* cfg, const void* workspace, size_t ws_b
 size_t mla_combine_out_proj_workspace_size(const mla_config* cfg, int32_t batch, int32_t n_q) {
   if (check_cfg(cfg) != MLA_OK || batch < 0 || n_q <= 0 || cfg->dtype != MLA_BF16 || !proj_tc_supported(cfg))
     return 0;
+  if ((long long)batch * n_q > kPlanMaxRows) return 0;
+  // the merge takes up to ocomb::kMaxN segments (rows plus the plan's extra cuts) in one launch
+  const DecodeLayout L = decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, 0),
+                                       qpack_row_bytes(cfg), part_elem(cfg));
+  if (!pairdec::supports(cfg) || !ocomb::supports(cfg, L.max_segments)) return 0;
   const int n = batch * n_q;
   const ProjSpecs ps = proj_specs(cfg, n, false, nullptr, nullptr, nullptr, nullptr, nullptr, kSizeOnly, kSizeOnly,
                                   kSizeOnly, kSizeOnly, kSizeOnly, kSizeOnly, kSizeOnly);

@@ -142,6 +142,12 @@ WORKLOADS: Dict[str, Workload] = {
         "v3_b128_nq2_ragged512_16k", SHAPES["v3"], batch=128, n_q=2, len_lo=512, len_hi=16384,
         description="V3-shaped multi-token decode, batch 128, 2 causal query tokens per sequence, "
                     "ragged lengths U[512, 16384], append 2 rows then attend"),
+    "v3_prefill_b8_c64_ragged1k_4k": Workload(
+        "v3_prefill_b8_c64_ragged1k_4k", SHAPES["v3"], batch=8, n_q=64, len_lo=1024, len_hi=4096,
+        shuffled_blocks=True,
+        description="V3-shaped chunked prefill over the latent cache, batch 8, a 64-token chunk per "
+                    "sequence (appended, then each token attends causally), ragged cached lengths "
+                    "U[1024, 4096], 64-token pages in shuffled order"),
 }
 
 

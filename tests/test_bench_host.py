@@ -80,3 +80,21 @@ def test_reference_arm_reports_the_gpu_arms_metric(bench):
     import inspect
     src = inspect.getsource(bench.run_reference) + inspect.getsource(bench.run_ours)
     assert src.count('"metric": METRIC') == 2
+
+
+def test_decode_roofline_counts_causal_rows_and_picks_the_larger_floor(bench):
+    import torch
+    from mla_synth import WORKLOADS, generate, reduced
+    peaks = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+    for n_q, bound in ((1, "hbm"), (64, "tensor")):
+        wl = reduced(WORKLOADS["v3_prefill_b8_c64_ragged1k_4k"], lengths=[0, 5, 300], n_q=n_q)
+        data = generate(wl)
+        # visible rows, one query row at a time: sequence b's row j sees L_b + j + 1 rows
+        visible = sum(int(data.cached_len[b]) + j + 1 for b in range(wl.batch) for j in range(n_q))
+        sh = wl.shape
+        assert bench.decode_flops(wl, data) == visible * (2 * sh.n_heads * (2 * sh.d_c + sh.d_r))
+        cache = int(data.seq_lens.sum()) * sh.row * sh.elem_bytes
+        r = bench.decode_roofline(wl, data, cache, 1e-4, peaks, None)
+        assert r["bound"] == bound
+        floor = max(r["hbm_floor_us"], r["tensor_floor_us"]) if bound == "tensor" else r["hbm_floor_us"]
+        assert abs(r["frac"] - floor / 100.0) < 1e-9

@@ -44,6 +44,8 @@ SMALL_CASES = [
     ("v3_b128_nq2_ragged512_16k", [0, 1, 62, 63, 64, 300], 2),
     # 260 new tokens: the projections run in two token chunks
     ("v3_b128_nq2_ragged512_16k", [3] * 130, 2),
+    # chunked prefill: 16 causal query tokens per sequence, one with an empty cache
+    ("v3_prefill_b8_c64_ragged1k_4k", [0, 65, 200], 16),
 ]
 
 
@@ -59,7 +61,8 @@ def test_small_cases_every_element(name, lengths, n_q):
     check_outputs(layer, data, exp, range(wl.n_tok))
 
 
-FULL = ["v2_b16_l4096", "v3_b64_ragged1k_8k", "v3_b4_long", "v3_b128_nq2_ragged512_16k"]
+FULL = ["v2_b16_l4096", "v3_b64_ragged1k_8k", "v3_b4_long", "v3_b128_nq2_ragged512_16k",
+        "v3_prefill_b8_c64_ragged1k_4k"]
 
 
 @pytest.mark.parametrize("name", FULL)

@@ -246,7 +246,7 @@ BRUTE_SHAPE_Q = MLAShape("brute_q", hidden=7, n_heads=3, d_c=4, d_r=2, qk_nope=2
                          q_lora=3, rope_theta=20.0, dtype="bf16")
 
 
-@pytest.mark.parametrize("n_q,shape", [(1, BRUTE_SHAPE), (2, BRUTE_SHAPE), (2, BRUTE_SHAPE_Q)])
+@pytest.mark.parametrize("n_q,shape", [(1, BRUTE_SHAPE), (2, BRUTE_SHAPE), (2, BRUTE_SHAPE_Q), (5, BRUTE_SHAPE)])
 def test_oracle_matches_brute_force_loops(n_q, shape):
     rng = np.random.default_rng(10 + n_q)
     W = {k: rng.standard_normal(s) / math.sqrt(s[0]) for k, s in shape.weight_shapes().items()}
