@@ -42,8 +42,12 @@ def needs_build() -> bool:
 
 
 def command(out: Path = LIB, extra=()):
+    # -fno-gnu-unique: the per-kernel "attribute already set" statics of the
+    # launchers stay private to each loaded copy of the library (two builds in
+    # one process would otherwise share them and skip each other's setup).
     return [_nvcc(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "-shared",
-            "-Xcompiler", "-fPIC", "-Xptxas", "-warn-spills", f"-I{INCLUDE}", f"-I{CSRC}",
+            "-Xcompiler", "-fPIC", "-Xcompiler", "-fno-gnu-unique", "-Xptxas", "-warn-spills",
+            f"-I{INCLUDE}", f"-I{CSRC}",
             *extra, "-o", str(out), str(CSRC / "mla_abi.cu")]
 
 

@@ -14,6 +14,7 @@
 #include "elementwise.cuh"
 #include "gemm_simt.cuh"
 #include "out_combine.cuh"
+#include "qhead_tc.cuh"
 #include "wgemm_tc.cuh"
 
 using namespace mla;
@@ -187,6 +188,9 @@ mla_status out_impl(const mla_config* c, const float* o_lat, int n, const void* 
   return MLA_OK;
 }
 
+// Time limit of every bounded wait in the tensor-core kernels (process-wide).
+std::atomic<unsigned long long> g_wait_limit_ns{sm100::kWaitLimitNs};
+
 // ---------------------------------------------------------------- bf16 projections
 // Tensor-core path of the query and output projections (weights bf16; see
 // wgemm_tc.cuh).  Activations enter the MMAs in bf16; with the split-query
@@ -264,9 +268,15 @@ mla_status absorb_tc(const mla_config* c, const void* x, int n, const void* W_DQ
   const ProjSpecs ps = proj_specs(c, n, split, W_DQ, W_UQ, W_UK, nullptr, nullptr, static_cast<const bf16*>(x),
                                   cq_hi, cq_lo, qn_hi, qn_lo, nullptr, nullptr);
   if (c->q_lora > 0) MLA_TRY(wg::run(ps.dq, part, nullptr, cq_hi, cq_lo, s));
-  MLA_TRY(wg::run(ps.uq, part, q_f, nullptr, nullptr, s));
   const int H = c->n_heads, nope = c->qk_nope, row = c->d_c + c->d_r;
   bf16* qp_lo = q_packed && split ? q_packed + (long long)n * H * row : nullptr;
+  if (qh::supports(c, n)) {  // W_UQ head slice, RoPE and W_UK in one kernel (rotation table in the q_f region)
+    static_assert(sizeof(double) * 64 <= 4 * 192, "rotation table larger than the fp32 query it replaces");
+    return qh::launch(c, n, cq_hi, cq_lo, static_cast<const bf16*>(W_UQ), static_cast<const bf16*>(W_UK), pos,
+                      reinterpret_cast<double*>(q_f), q_packed, qp_lo, q_packed ? nullptr : q_lat,
+                      q_packed ? nullptr : q_rope, g_wait_limit_ns.load(std::memory_order_relaxed), s);
+  }
+  MLA_TRY(wg::run(ps.uq, part, q_f, nullptr, nullptr, s));
   const dim3 qgrid(n, (H + kHeadGroup - 1) / kHeadGroup);
   MLA_CUDA(launch_chained(query_split_bf16_kernel, qgrid, dim3(256), sizeof(double) * c->d_r, s, (const float*)q_f, n, H,
                           nope, c->d_r, c->rope_theta, pos, qn_hi, qn_lo, q_rope, q_packed, qp_lo, row, c->d_c));
@@ -328,8 +338,6 @@ size_t qpack_row_bytes(const mla_config* c) {
 // (they feed bf16 MMAs next), fp32 from the CUDA-core one.
 int part_elem(const mla_config* c) { return c->dtype == MLA_BF16 ? 2 : 4; }
 
-// Time limit of every bounded wait in the tensor-core decode (process-wide).
-std::atomic<unsigned long long> g_wait_limit_ns{sm100::kWaitLimitNs};
 
 int resolve_workers(const mla_config* c, int max_workers) {
   return max_workers > 0 ? max_workers : default_workers(c);

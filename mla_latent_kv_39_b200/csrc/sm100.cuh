@@ -122,12 +122,11 @@ __device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity) {
   return kCluster ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity);
 }
 
-// `sleep_ns` > 0 backs off between polls (for roles that wait long while
-// other warps of the SM issue work).
-template <bool kCluster = false>
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int where,
-                                          uint64_t limit_ns = kWaitLimitNs, uint32_t sleep_ns = 0) {
-  if (mbar_poll<kCluster>(bar, parity)) return true;
+// The polling loop of a wait that did not complete at once, out of line: a
+// kernel with many wait sites keeps one copy of it (instruction cache).
+template <bool kCluster>
+__device__ __noinline__ bool mbar_wait_loop(uint64_t* bar, uint32_t parity, int where, uint64_t limit_ns,
+                                            uint32_t sleep_ns) {
   const uint64_t t0 = global_ns();
   for (uint32_t it = 0;; ++it) {
     if (sleep_ns) __nanosleep(sleep_ns);
@@ -137,6 +136,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int wh
       return false;
     }
   }
+}
+
+// `sleep_ns` > 0 backs off between polls (for roles that wait long while
+// other warps of the SM issue work).
+template <bool kCluster = false>
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int where,
+                                          uint64_t limit_ns = kWaitLimitNs, uint32_t sleep_ns = 0) {
+  if (mbar_poll<kCluster>(bar, parity)) return true;
+  return mbar_wait_loop<kCluster>(bar, parity, where, limit_ns, sleep_ns);
 }
 
 // ------------------------------------------------------------------ proxies
@@ -152,6 +160,36 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
       ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// 3-D tile load (no cluster broadcast), like tma_load_2d.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// 3-D tile store: this CTA's shared-memory box to coordinates (x, y, z) of
+// the tensor map (elements outside the tensor are not written), tracked by
+// this thread's bulk-async groups.  The writes that filled `src` must be made
+// visible to the async proxy first (fence_proxy_async_smem + a barrier).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(map), "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until every committed bulk store of this thread has read its shared
+// memory (the source may then be reused or released).
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Pull a tile of a 2-D tensor map into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void prefetch_l2_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
 }
 
 // Pull a tile of a 3-D tensor map into L2 (no shared memory, no barrier).

@@ -69,13 +69,6 @@ struct Params {
   long long o_ts, o_gs;  // output element (t, g, f) at t o_ts + g o_gs + f
 };
 
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
-      ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-
 // Work item -> (group, feature tile, K split).  Consecutive items (which run
 // on consecutive CTAs at about the same time) take neighbouring columns of the
 // weight matrix for the same K rows, so together they read whole DRAM pages
@@ -95,11 +88,6 @@ __device__ __forceinline__ void item_coords(const Params& p, int item, int& g, i
   }
   kb0 = (int)((long long)s * p.KB / p.S);
   kb1 = (int)((long long)(s + 1) * p.KB / p.S);
-}
-
-__device__ __forceinline__ void prefetch_l2_2d(const CUtensorMap* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
-               : "memory");
 }
 
 __device__ __forceinline__ void set_abort(Smem& sm) { *(volatile int*)&sm.abort_flag = 1; }
