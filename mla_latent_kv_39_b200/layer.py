@@ -154,6 +154,21 @@ class DecodeLayer:
         self.project(stream)
         return self.y
 
+    def capture_step(self, x, seq_idx, pos, seq_lens, want_o_lat: bool = False) -> torch.cuda.CUDAGraph:
+        """Record one ``step`` on these device buffers as a CUDA graph: the
+        launches (and the side-stream fork and join) are replayed by
+        ``graph.replay()`` without host work.  Refill ``x``, ``seq_idx``,
+        ``pos`` and ``seq_lens`` in place between replays; ``self.y`` holds the
+        result.  One eager step runs first (outside the capture) so that every
+        kernel's one-time setup is done; it appends the same rows the replays
+        append again."""
+        self.step(x, seq_idx, pos, seq_lens, want_o_lat=want_o_lat)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.step(x, seq_idx, pos, seq_lens, want_o_lat=want_o_lat)
+        return graph
+
     def run_from_host(self, inputs, y_hosts, between=None, stream=None, copy_stream=None):
         """Several steps over host (pinned) inputs, pipelined.
 

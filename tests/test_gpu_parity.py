@@ -248,3 +248,32 @@ def test_plan_on_the_side_stream_gives_the_same_result():
     check_device_error()
     assert torch.equal(layer.o_lat, o_a)
     assert torch.equal(layer.y, y_a)
+
+
+def test_graph_replay_of_the_step_matches_the_eager_step():
+    """capture_step records the whole step (fork to the side stream and join
+    included); replays give the eager step's y and o_lat, also after the
+    inputs are refilled in place."""
+    wl = reduced(WORKLOADS["v3_b64_ragged1k_8k"], lengths=[700, 64, 1, 130])
+    data, dev, layer = run_gpu(wl)
+    x, si, pos, sl = dev["x_new"], dev["seq_idx"], dev["pos"], dev["seq_lens"]
+    y_eager, o_eager = layer.y.clone(), layer.o_lat.clone()
+    graph = layer.capture_step(x, si, pos, sl, want_o_lat=True)
+    layer.y.zero_()
+    layer.o_lat.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    check_device_error()
+    assert torch.equal(layer.y, y_eager)
+    assert torch.equal(layer.o_lat, o_eager)
+    # new hidden states for the same positions: replay == eager
+    x.copy_(torch.flip(x, dims=[1]))
+    graph.replay()
+    torch.cuda.synchronize()
+    y_graph, o_graph = layer.y.clone(), layer.o_lat.clone()
+    layer.step(x, si, pos, sl, want_o_lat=True)
+    torch.cuda.synchronize()
+    check_device_error()
+    assert not torch.equal(y_graph, y_eager)
+    assert torch.equal(layer.y, y_graph)
+    assert torch.equal(layer.o_lat, o_graph)
