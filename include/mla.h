@@ -201,7 +201,9 @@ mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok,
  *            from mla_absorb_q (row v = b n_q + j)
  *   seq_lens int32 [batch]: rows of each sequence INCLUDING the n_q new rows
  *            (already appended); must satisfy n_q <= seq_lens[b] <=
- *            max_blocks_per_seq * block_size.
+ *            max_blocks_per_seq * block_size, or seq_lens[b] = 0: an empty
+ *            sequence (a shard without rows of it, see mla_merge_shards),
+ *            whose query rows get o_lat = 0 and lse = -inf.
  *   max_workers: upper bound on parallel workers (0 = sized to the device).
  *   workspace >= mla_decode_workspace_size(cfg, batch, n_q, max_workers)
  * Device errors: bad lengths or block ids -> MLA_ERR_BOUNDS (that sequence's
@@ -273,6 +275,36 @@ mla_status mla_decode_packed_planned(const mla_config* cfg, const void* q_packed
  * ------------------------------------------------------------------------- */
 mla_status mla_combine(const mla_config* cfg, const void* workspace, size_t ws_bytes,
                        int32_t batch, int32_t n_q, float* o_lat, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Sequence split across GPUs (not on the pages: the step-4a merge one level
+ * up, for contexts too long for one GPU's cache or time budget).  The cached
+ * pages of a sequence are cut into contiguous page ranges ("shards") held by
+ * different GPUs.  Each GPU decodes its shard (its own cache and block-table
+ * rows, the shard's number of visible rows as seq_lens, n_q = 1 per query
+ * row), takes per-row (o_lat, lse) with mla_combine_lse, the pairs of all
+ * shards are exchanged (e.g. an all-gather over NVLink), and
+ * mla_merge_shards merges them:
+ *   o[t,h] = sum_r 2^(lse_r - M) o_r / sum_r 2^(lse_r - M),  M = max_r lse_r
+ *   lse[t,h] = M + log2 sum_r 2^(lse_r - M)
+ * which equals the decode over the whole key set up to fp32 rounding.
+ *   mla_combine_lse: mla_combine, plus
+ *     lse      float32 [batch n_q, H] (out): the base-2 log-sum-exp of the
+ *              scaled scores (scale log2 e) over the keys decoded; -inf for a
+ *              row with no key (its o_lat is then 0).
+ *   mla_merge_shards:
+ *     o_parts  float32 [n_shards, rows, H, d_c] (in), 16-byte aligned
+ *     lse_parts float32 [n_shards, rows, H] (in)
+ *     o_lat    float32 [rows, H, d_c] (out), 16-byte aligned
+ *     lse      float32 [rows, H] (out, may be NULL)
+ *   A row whose shards all have lse = -inf gets o = 0, lse = -inf.
+ * Errors: MLA_ERR_INVALID_ARG for NULL / misaligned pointers or counts < 0
+ * (n_shards < 1); MLA_ERR_UNSUPPORTED for d_c not a multiple of 8 or > 2048.
+ * ------------------------------------------------------------------------- */
+mla_status mla_combine_lse(const mla_config* cfg, const void* workspace, size_t ws_bytes,
+                           int32_t batch, int32_t n_q, float* o_lat, float* lse, void* stream);
+mla_status mla_merge_shards(const mla_config* cfg, int32_t n_shards, int32_t rows, const float* o_parts,
+                            const float* lse_parts, float* o_lat, float* lse, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Step 4b - output side with W_UV absorbed ([P5] section 1 "Định nghĩa":

@@ -18,6 +18,7 @@ from .abi import (  # noqa: F401
     mla_cache_append_workspace_size,
     mla_cache_append_noalloc,
     mla_combine,
+    mla_combine_lse,
     mla_combine_out_proj,
     mla_combine_out_proj_workspace_size,
     mla_decode,
@@ -27,8 +28,10 @@ from .abi import (  # noqa: F401
     mla_decode_workspace_size,
     mla_get_device_error,
     mla_kernel_launches,
+    mla_merge_shards,
     mla_out_proj,
     mla_out_proj_workspace_size,
     mla_query_packed_bytes,
 )
 from .layer import DecodeLayer  # noqa: F401
+from .shard import ShardPlan, decode_shard, decode_sharded, gather_partials, shard_plan  # noqa: F401

@@ -71,6 +71,8 @@ SIGNATURES = {
     "mla_decode_workspace_size": (_sz, [_P_CFG, _i32, _i32, _i32]),
     "mla_decode": (_i32, [_P_CFG, _vp, _vp, _i32, _i32, _P_CACHE, _vp, _i32, _vp, _sz, _vp]),
     "mla_combine": (_i32, [_P_CFG, _vp, _sz, _i32, _i32, _vp, _vp]),
+    "mla_combine_lse": (_i32, [_P_CFG, _vp, _sz, _i32, _i32, _vp, _vp, _vp]),
+    "mla_merge_shards": (_i32, [_P_CFG, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "mla_combine_out_proj_workspace_size": (_sz, [_P_CFG, _i32, _i32]),
     "mla_combine_out_proj": (_i32, [_P_CFG, _vp, _sz, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mla_out_proj_workspace_size": (_sz, [_P_CFG, _i32]),
@@ -338,6 +340,26 @@ def mla_combine(cfg: Config, workspace, batch: int, n_q: int, o_lat, stream=None
     _need(o_lat, "o_lat", torch.float32, shape=(batch * n_q, cfg.n_heads, cfg.d_c))
     _check(lib().mla_combine(ctypes.byref(cfg.c()), _ptr(workspace), workspace.numel(), batch, n_q,
                              _ptr(o_lat), _stream(stream)), "mla_combine")
+
+
+def mla_combine_lse(cfg: Config, workspace, batch: int, n_q: int, o_lat, lse, stream=None):
+    _need(workspace, "workspace", torch.uint8)
+    _need(o_lat, "o_lat", torch.float32, shape=(batch * n_q, cfg.n_heads, cfg.d_c))
+    _need(lse, "lse", torch.float32, shape=(batch * n_q, cfg.n_heads))
+    _check(lib().mla_combine_lse(ctypes.byref(cfg.c()), _ptr(workspace), workspace.numel(), batch, n_q,
+                                 _ptr(o_lat), _ptr(lse), _stream(stream)), "mla_combine_lse")
+
+
+def mla_merge_shards(cfg: Config, o_parts, lse_parts, o_lat, lse=None, stream=None):
+    """``o_parts`` [S, rows, H, d_c], ``lse_parts`` [S, rows, H] -> ``o_lat`` [rows, H, d_c] (+ ``lse``)."""
+    _need(o_parts, "o_parts", torch.float32, ndim=4)
+    S, rows = o_parts.shape[0], o_parts.shape[1]
+    _need(lse_parts, "lse_parts", torch.float32, shape=(S, rows, cfg.n_heads))
+    _need(o_lat, "o_lat", torch.float32, shape=(rows, cfg.n_heads, cfg.d_c))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, shape=(rows, cfg.n_heads))
+    _check(lib().mla_merge_shards(ctypes.byref(cfg.c()), S, rows, _ptr(o_parts), _ptr(lse_parts), _ptr(o_lat),
+                                  _ptr(lse), _stream(stream)), "mla_merge_shards")
 
 
 def mla_combine_out_proj_workspace_size(cfg: Config, batch: int, n_q: int) -> int:

@@ -3,7 +3,7 @@
 // The unit of work is a query row v = b * n_q + j (query j of sequence b).
 // Row v sees the cache rows 0 .. len_v - 1 of sequence b, with
 // len_v = seq_lens[b] - n_q + j + 1 (causal, its own row included), i.e.
-// ceil(len_v / block) pages.  The pages of all query rows, laid end to end,
+// ceil(len_v / block) pages (none for an empty sequence, seq_lens[b] = 0).  The pages of all query rows, laid end to end,
 // are cut into `workers` contiguous ranges of about equal cost (pages plus a
 // fixed charge per row for the segment's setup); where a range crosses a row
 // boundary it is cut again, so every piece - a "segment" - covers pages
@@ -143,7 +143,9 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ seq_lens, 
   auto pages_of = [&](int v) -> int {
     const int b = v / n_q, j = v % n_q;
     const int len = seq_lens[b];
-    if (len < n_q || len > max_blocks * bs) {
+    // 0: an empty sequence (e.g. a shard of another GPU's pages holding none
+    // of this one's), whose query rows see no row
+    if (len < 0 || (len > 0 && len < n_q) || len > max_blocks * bs) {
       if (j == 0) report(MLA_ERR_BOUNDS, 4, b, len);
       return 0;
     }
@@ -229,15 +231,18 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const int32_t* __rest
 // Weight of segment `first + s` in the merge of query row v for head h:
 // 2^(lse_s - M) / sum_s' 2^(lse_s' - M) with M the largest lse of the row.
 struct RowMerge {
-  float M, invZ;
-  __device__ RowMerge(const float* lse, int first, int n, int H, int h) : M(-INFINITY), invZ(0.f) {
-    for (int s = 0; s < n; ++s) M = fmaxf(M, lse[(long long)(first + s) * H + h]);
+  float M, Z, invZ;
+  // the n log2-sum-exps at lse[(first + s) * stride + h], s < n
+  __device__ RowMerge(const float* lse, long long first, int n, long long stride, int h)
+      : M(-INFINITY), Z(0.f), invZ(0.f) {
+    for (int s = 0; s < n; ++s) M = fmaxf(M, lse[(first + s) * stride + h]);
     if (M == -INFINITY) return;
-    float Z = 0.f;
-    for (int s = 0; s < n; ++s) Z += exp2f(lse[(long long)(first + s) * H + h] - M);
+    for (int s = 0; s < n; ++s) Z += exp2f(lse[(first + s) * stride + h] - M);
     invZ = 1.f / Z;
   }
   __device__ float weight(float lse_s) const { return invZ > 0.f ? exp2f(lse_s - M) * invZ : 0.f; }
+  // log2-sum-exp of the merged pieces (-inf when none holds a key)
+  __device__ float lse() const { return M == -INFINITY ? -INFINITY : M + log2f(Z); }
 };
 
 __device__ __forceinline__ void load8(const float* p, float (&x)[8]) {
@@ -261,7 +266,7 @@ __device__ __forceinline__ void load8(const bf16* p, float (&x)[8]) {
 // With `valid` false (a workspace no decode wrote) the row is written as zeros.
 template <typename P>
 __device__ void combine_rows(const void* ws, const DecodeLayout& L, bool valid, int v, int H, int d_c,
-                             float* __restrict__ o_lat) {
+                             float* __restrict__ o_lat, float* __restrict__ lse_out) {
   const int per_head = d_c / 8;
   const int hb = blockDim.x / per_head;
   const int h = blockIdx.y * hb + threadIdx.x / per_head, d0 = 8 * (threadIdx.x % per_head);
@@ -271,6 +276,7 @@ __device__ void combine_rows(const void* ws, const DecodeLayout& L, bool valid, 
   const float* lse = ws_at<float>(ws, L.off_lse);
   const P* part = ws_at<P>(ws, L.off_o);
   const RowMerge rm(lse, first, n, H, h);
+  if (lse_out != nullptr && d0 == 0) lse_out[(long long)v * H + h] = rm.lse();
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   for (int s = 0; s < n; ++s) {
     const float w = rm.weight(lse[(long long)(first + s) * H + h]);
@@ -286,7 +292,7 @@ __device__ void combine_rows(const void* ws, const DecodeLayout& L, bool valid, 
 }
 
 __global__ void __launch_bounds__(256) combine_kernel(const void* ws, long long ws_bytes, int batch, int n_q, int H,
-                                                      int d_c, float* __restrict__ o_lat) {
+                                                      int d_c, float* __restrict__ o_lat, float* __restrict__ lse_out) {
   pdl_wait();
   pdl_trigger();
   const DecodeHeader* hd = ws_at<DecodeHeader>(ws, 0);
@@ -295,8 +301,41 @@ __global__ void __launch_bounds__(256) combine_kernel(const void* ws, long long 
   const int v = blockIdx.x;
   if (bad && v == 0 && blockIdx.y == 0 && threadIdx.x == 0) report(MLA_ERR_WORKSPACE, 0, batch, n_q);
   const DecodeLayout L = hd->layout;
-  if (!bad && L.part_elem == 2) combine_rows<bf16>(ws, L, true, v, H, d_c, o_lat);
-  else combine_rows<float>(ws, L, !bad, v, H, d_c, o_lat);
+  if (!bad && L.part_elem == 2) combine_rows<bf16>(ws, L, true, v, H, d_c, o_lat, lse_out);
+  else combine_rows<float>(ws, L, !bad, v, H, d_c, o_lat, lse_out);
+}
+
+// The same merge one level up: o_parts[r] and lse_parts[r] are the
+// (o_lat, log2-sum-exp) of query rows over shard r of every sequence's keys
+// (e.g. the pages held by GPU r), all shards of a row together are its whole
+// key set.  o_lat[v, h] = sum_r 2^(lse_r - M) o_r / sum_r 2^(lse_r - M), and
+// lse_out (optional) the merged log2-sum-exp.  Grid and threads as combine.
+__global__ void __launch_bounds__(256) merge_shards_kernel(const float* __restrict__ o_parts,
+                                                           const float* __restrict__ lse_parts, int n_shards,
+                                                           int rows, int H, int d_c, float* __restrict__ o_lat,
+                                                           float* __restrict__ lse_out) {
+  pdl_wait();
+  pdl_trigger();
+  const int per_head = d_c / 8;
+  const int hb = blockDim.x / per_head;
+  const int v = blockIdx.x;
+  const int h = blockIdx.y * hb + threadIdx.x / per_head, d0 = 8 * (threadIdx.x % per_head);
+  if (h >= H || threadIdx.x >= hb * per_head) return;
+  const long long stride = (long long)rows * H;  // between shards, in lse entries
+  const RowMerge rm(lse_parts, 0, n_shards, stride, v * H + h);
+  if (lse_out != nullptr && d0 == 0) lse_out[(long long)v * H + h] = rm.lse();
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int r = 0; r < n_shards; ++r) {
+    const float w = rm.weight(lse_parts[r * stride + (long long)v * H + h]);
+    if (w == 0.f) continue;  // a shard without keys for this row
+    float x[8];
+    load8(o_parts + (r * stride + (long long)v * H + h) * d_c + d0, x);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = fmaf(w, x[k], acc[k]);
+  }
+  float* out = o_lat + ((long long)v * H + h) * d_c + d0;
+  *reinterpret_cast<float4*>(out) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  *reinterpret_cast<float4*>(out + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
 }
 
 }  // namespace mla

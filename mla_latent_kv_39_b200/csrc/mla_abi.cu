@@ -415,6 +415,25 @@ __global__ void wait_timeout_check_kernel(unsigned long long limit_ns) {
 
 }  // namespace
 
+namespace {
+mla_status combine_impl(const mla_config* cfg, const void* workspace, size_t ws_bytes, int32_t batch, int32_t n_q,
+                        float* o_lat, float* lse, void* stream) {
+  MLA_TRY(check_cfg(cfg));
+  if (batch < 0 || n_q <= 0) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!workspace || !o_lat) return MLA_ERR_INVALID_ARG;
+  if (ws_bytes < sizeof(DecodeHeader)) return MLA_ERR_WORKSPACE;
+  if (!all_aligned16(workspace, o_lat)) return MLA_ERR_INVALID_ARG;
+  if (lse != nullptr && ((uintptr_t)lse & 3u)) return MLA_ERR_INVALID_ARG;
+  if (cfg->d_c % 8 != 0 || cfg->d_c / 8 > 256) return MLA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int per_head = cfg->d_c / 8, heads_per_block = 256 / per_head;
+  dim3 grid(batch * n_q, (cfg->n_heads + heads_per_block - 1) / heads_per_block);
+  return st(launch_chained(combine_kernel, grid, dim3(256), 0, s, (const void*)workspace, (long long)ws_bytes, batch,
+                            n_q, cfg->n_heads, cfg->d_c, o_lat, lse));
+}
+}  // namespace
+
 extern "C" {
 
 int32_t mla_abi_version(void) { return MLA_ABI_VERSION; }
@@ -615,18 +634,29 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
 
 mla_status mla_combine(const mla_config* cfg, const void* workspace, size_t ws_bytes, int32_t batch,
                        int32_t n_q, float* o_lat, void* stream) {
+  return combine_impl(cfg, workspace, ws_bytes, batch, n_q, o_lat, nullptr, stream);
+}
+
+mla_status mla_combine_lse(const mla_config* cfg, const void* workspace, size_t ws_bytes, int32_t batch,
+                           int32_t n_q, float* o_lat, float* lse, void* stream) {
+  if (lse == nullptr) return MLA_ERR_INVALID_ARG;
+  return combine_impl(cfg, workspace, ws_bytes, batch, n_q, o_lat, lse, stream);
+}
+
+mla_status mla_merge_shards(const mla_config* cfg, int32_t n_shards, int32_t rows, const float* o_parts,
+                            const float* lse_parts, float* o_lat, float* lse, void* stream) {
   MLA_TRY(check_cfg(cfg));
-  if (batch < 0 || n_q <= 0) return MLA_ERR_INVALID_ARG;
-  if (batch == 0) return MLA_OK;
-  if (!workspace || !o_lat) return MLA_ERR_INVALID_ARG;
-  if (ws_bytes < sizeof(DecodeHeader)) return MLA_ERR_WORKSPACE;
-  if (!all_aligned16(workspace, o_lat)) return MLA_ERR_INVALID_ARG;
+  if (n_shards <= 0 || rows < 0) return MLA_ERR_INVALID_ARG;
+  if (rows == 0) return MLA_OK;
+  if (!o_parts || !lse_parts || !o_lat) return MLA_ERR_INVALID_ARG;
+  if (!all_aligned16(o_parts, o_lat) || ((uintptr_t)lse_parts & 3u) || (lse != nullptr && ((uintptr_t)lse & 3u)))
+    return MLA_ERR_INVALID_ARG;
   if (cfg->d_c % 8 != 0 || cfg->d_c / 8 > 256) return MLA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int per_head = cfg->d_c / 8, heads_per_block = 256 / per_head;
-  dim3 grid(batch * n_q, (cfg->n_heads + heads_per_block - 1) / heads_per_block);
-  return st(launch_chained(combine_kernel, grid, dim3(256), 0, s, (const void*)workspace, (long long)ws_bytes, batch,
-                            n_q, cfg->n_heads, cfg->d_c, o_lat));
+  dim3 grid(rows, (cfg->n_heads + heads_per_block - 1) / heads_per_block);
+  return st(launch_chained(merge_shards_kernel, grid, dim3(256), 0, s, o_parts, lse_parts, (int)n_shards, (int)rows,
+                            cfg->n_heads, cfg->d_c, o_lat, lse));
 }
 
 size_t mla_combine_out_proj_workspace_size(const mla_config* cfg, int32_t batch, int32_t n_q) {
