@@ -115,6 +115,8 @@ def decode_roofline(wl, data, cache_bytes: int, dec_s: float, peaks, traffic):
     hbm_s = cache_bytes / (peaks["hbm_gbs"] * 1e9)
     tensor_s = flops / (peaks["bf16_tflops"] * 1e12)
     kernel = "mla_decode_packed_planned call (the pair decode kernel; its split plan runs beside the query projections)"
+    if wl.fp8_cache:
+        kernel = "mla_decode call (CUDA-core decode of the E4M3 cache rows and their scales, plan included)"
     if wl.n_q > 1 and tensor_s > hbm_s:
         achieved = flops / dec_s / 1e12
         return {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -225,6 +227,8 @@ def oracle_sample(wl, budget_s: float = 15.0, max_seqs: int = 64, data=None, W=N
         rows = oracle.to64(data.cached_rows[s:e]) if data.cached_rows is not None else None
         toks = slice(b * wl.n_q, (b + 1) * wl.n_q)
         t0 = time.perf_counter()
+        if wl.fp8_cache:      # the values the stored E4M3 codes and row scales stand for
+            rows = oracle.e4m3_value(data.cached_codes[s:e].numpy()) * oracle.to64(data.cached_scale[s:e])[:, None]
         if rows is None:
             c, kr = oracle.latent_rows(data.x_cached[s:e], W["W_DKV"], W["W_KR"], np.arange(e - s),
                                        shape.rope_theta, shape.dtype)
@@ -232,7 +236,7 @@ def oracle_sample(wl, budget_s: float = 15.0, max_seqs: int = 64, data=None, W=N
             c, kr = rows[:, :shape.d_c], rows[:, shape.d_c:]
         pos = data.new_positions().numpy()[toks]
         oracle.decode_step(shape, W, oracle.to64(data.x_new[toks]), pos, [c], [kr], wl.n_q,
-                           order="decompressed")
+                           order="decompressed", cache_dtype="fp8" if wl.fp8_cache else None)
         t_spent += time.perf_counter() - t0
         done_tok += wl.n_q
         seqs += 1
@@ -313,8 +317,8 @@ def run_ours(args):
     wl = dataclasses.replace(base, seed=rank_seed(base.seed, rank))
     data = generate(wl)
     dev = device_inputs(data, device)
-    cfg = mla.Config.from_shape(wl.shape, split_query=wl.split_query)
-    cache = mla.Cache(dev["pool"], dev["block_table"])
+    cfg = mla.Config.from_shape(wl.shape, split_query=wl.split_query, fp8_cache=wl.fp8_cache)
+    cache = mla.Cache(dev["pool"], dev["block_table"], dev["row_scale"])
     layer = mla.DecodeLayer(cfg, dev["weights"], cache, wl.batch, wl.n_q, args.max_workers)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     clean = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
@@ -417,7 +421,7 @@ def run_ours(args):
     mla.check_device_error()
 
     peaks = measured_peaks()
-    cache_bytes = int(data.seq_lens.sum()) * wl.shape.row * wl.shape.elem_bytes
+    cache_bytes = int(data.seq_lens.sum()) * wl.cache_row_bytes
     dec_avg_s = statistics.mean(dec_ms) / 1000.0
     achieved = cache_bytes / dec_avg_s / 1e9
     traffic = recorded_traffic(wl.name)
@@ -444,7 +448,8 @@ def run_ours(args):
                    "cache_rows": int(data.seq_lens.sum()), "block_size": wl.shape.block_size,
                    "page_order": "shuffled" if wl.shuffled_blocks else "in order",
                    "l2": "flushed before every step outside the timed events (256 MiB write, then a 256 MiB read)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "cache_format": "e4m3 codes + fp32 row scale" if wl.fp8_cache else wl.shape.dtype},
         "latent_kv_gbs": achieved,
         "decode_ms": statistics.mean(dec_ms),
         "step_ms_percentiles": percentiles(step_ms),

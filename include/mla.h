@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 1
+#define MLA_ABI_VERSION 2
 
 typedef enum {
   MLA_OK = 0,
@@ -97,10 +97,27 @@ typedef struct {
  * Costs extra score work in the bf16 decode kernel; no effect on fp32 storage. */
 #define MLA_FLAG_SPLIT_QUERY 1
 
+/* Latent cache in FP8 (OCP E4M3: 4 exponent bits, bias 7, 3 mantissa bits,
+ * largest finite 448) with one fp32 scale per cached row ([P2] "MLA ve diğer
+ * optimizasyonlarla ilişkisi": quantization is orthogonal to MLA and used
+ * together with it; the pages fix no format, this is the plainest per-row
+ * one).  A stored row [c_KV | k_R] stands for codes * scale with
+ *   scale = fp32(max_i |row_i| / 448)   (1 when that is 0),
+ *   code_i = E4M3(row_i / scale)        nearest, ties to even, from the exact
+ *                                       fp64 row; saturating at +-448.
+ * Requires dtype MLA_BF16 (weights and activations stay bf16) and
+ * mla_cache.row_scale.  A 576-value row takes 580 bytes instead of 1152.
+ * The decode of an FP8 cache runs on the CUDA-core path of mla_decode; the
+ * packed-query entry points return MLA_ERR_UNSUPPORTED for it. */
+#define MLA_FLAG_FP8_CACHE 2
+
 /* Paged latent cache of one layer ([P2] "MLA ve diğer optimizasyonlarla ilişkisi").
- * pool:        [num_blocks, block_size, d_c + d_r] storage dtype; row = [c_KV | k_R].
+ * pool:        [num_blocks, block_size, d_c + d_r] storage dtype (E4M3 codes,
+ *              one byte each, with MLA_FLAG_FP8_CACHE); row = [c_KV | k_R].
  * block_table: int32 [batch, max_blocks_per_seq]; entry (b, k) is the pool block
  *              holding positions [k*block_size, (k+1)*block_size) of sequence b.
+ * row_scale:   float32 [num_blocks, block_size], the scale of each row, with
+ *              MLA_FLAG_FP8_CACHE (4-byte aligned); NULL otherwise (ignored).
  * The library reads and writes the pool in place; the caller owns all of it. */
 typedef struct {
   void* pool;
@@ -108,6 +125,7 @@ typedef struct {
   const int32_t* block_table;
   int32_t batch;
   int32_t max_blocks_per_seq;
+  float* row_scale;
 } mla_cache;
 
 /* ---------------------------------------------------------------------------

@@ -29,6 +29,7 @@ MLA_ERR_WORKSPACE = -6
 MLA_F32 = 0
 MLA_BF16 = 1
 MLA_FLAG_SPLIT_QUERY = 1
+MLA_FLAG_FP8_CACHE = 2
 MLA_APPEND_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 # Every symbol the header declares, with (restype, argtypes).
@@ -48,7 +49,7 @@ class MLACache(ctypes.Structure):
     """Mirror of ``mla_cache``."""
 
     _fields_ = [("pool", _vp), ("num_blocks", _i32), ("block_table", _vp), ("batch", _i32),
-                ("max_blocks_per_seq", _i32)]
+                ("max_blocks_per_seq", _i32), ("row_scale", _vp)]
 
 
 _P_CFG = ctypes.POINTER(MLAConfig)
@@ -133,33 +134,44 @@ class Config:
     block_size: int = 64
     dtype: str = "bf16"
     split_query: bool = False
+    fp8_cache: bool = False       # E4M3 cache rows with one fp32 scale each (bf16 weights)
 
     @staticmethod
-    def from_shape(shape, split_query: bool = False) -> "Config":
+    def from_shape(shape, split_query: bool = False, fp8_cache: bool = False) -> "Config":
         return Config(shape.hidden, shape.n_heads, shape.d_c, shape.d_r, shape.qk_nope,
                       shape.v_head, shape.q_lora, float(shape.rope_theta), 0.0,
-                      shape.block_size, shape.dtype, split_query)
+                      shape.block_size, shape.dtype, split_query, fp8_cache)
 
     @property
     def torch_dtype(self) -> torch.dtype:
         return torch.bfloat16 if self.dtype == "bf16" else torch.float32
 
+    @property
+    def cache_torch_dtype(self) -> torch.dtype:
+        """Element type of the cache pool (uint8 E4M3 codes for an FP8 cache)."""
+        return torch.uint8 if self.fp8_cache else self.torch_dtype
+
     def c(self) -> MLAConfig:
         return MLAConfig(self.hidden, self.n_heads, self.d_c, self.d_r, self.qk_nope, self.v_head,
                          self.q_lora, self.rope_theta, self.softmax_scale, self.block_size,
                          MLA_BF16 if self.dtype == "bf16" else MLA_F32,
-                         MLA_FLAG_SPLIT_QUERY if self.split_query else 0)
+                         (MLA_FLAG_SPLIT_QUERY if self.split_query else 0)
+                         | (MLA_FLAG_FP8_CACHE if self.fp8_cache else 0))
 
 
 class Cache:
-    """A paged latent cache: pool ``[num_blocks, block, d_c + d_r]`` + block table."""
+    """A paged latent cache: pool ``[num_blocks, block, d_c + d_r]`` + block table
+    (+ ``row_scale`` float32 ``[num_blocks, block]`` for an FP8 pool of E4M3 codes)."""
 
-    def __init__(self, pool: torch.Tensor, block_table: torch.Tensor):
+    def __init__(self, pool: torch.Tensor, block_table: torch.Tensor, row_scale: Optional[torch.Tensor] = None):
         _need(pool, "pool", ndim=3)
         _need(block_table, "block_table", dtype=torch.int32, ndim=2)
-        self.pool, self.block_table = pool, block_table
+        if row_scale is not None:
+            _need(row_scale, "row_scale", dtype=torch.float32, shape=tuple(pool.shape[:2]))
+        self.pool, self.block_table, self.row_scale = pool, block_table, row_scale
         self.c = MLACache(pool.data_ptr(), pool.shape[0], block_table.data_ptr(),
-                          block_table.shape[0], block_table.shape[1])
+                          block_table.shape[0], block_table.shape[1],
+                          None if row_scale is None else row_scale.data_ptr())
 
 
 def _need(t: torch.Tensor, name: str, dtype=None, ndim=None, shape=None):
@@ -216,7 +228,7 @@ def mla_cache_append(cfg: Config, x, W_DKV, W_KR, seq_idx, pos, cache: Cache, wo
     _need(seq_idx, "seq_idx", torch.int32, shape=(n,))
     _need(pos, "pos", torch.int32, shape=(n,))
     _need(workspace, "workspace", torch.uint8)
-    if cache.pool.dtype != dt or cache.pool.shape[1:] != (cfg.block_size, cfg.d_c + cfg.d_r):
+    if cache.pool.dtype != cfg.cache_torch_dtype or cache.pool.shape[1:] != (cfg.block_size, cfg.d_c + cfg.d_r):
         raise ValueError("cache pool dtype/shape does not match the config")
     _check(lib().mla_cache_append(ctypes.byref(cfg.c()), _ptr(x), n, _ptr(W_DKV), _ptr(W_KR),
                                   _ptr(seq_idx), _ptr(pos), ctypes.byref(cache.c), _ptr(workspace),
@@ -234,7 +246,7 @@ def mla_cache_append_noalloc(cfg: Config, x, W_DKV, W_KR, seq_idx, pos, cache: C
     _need(W_KR, "W_KR", dt, shape=(cfg.hidden, cfg.d_r))
     _need(seq_idx, "seq_idx", torch.int32, shape=(n,))
     _need(pos, "pos", torch.int32, shape=(n,))
-    if cache.pool.dtype != dt or cache.pool.shape[1:] != (cfg.block_size, cfg.d_c + cfg.d_r):
+    if cache.pool.dtype != cfg.cache_torch_dtype or cache.pool.shape[1:] != (cfg.block_size, cfg.d_c + cfg.d_r):
         raise ValueError("cache pool dtype/shape does not match the config")
     _check(lib().mla_cache_append_noalloc(ctypes.byref(cfg.c()), _ptr(x), n, _ptr(W_DKV), _ptr(W_KR),
                                           _ptr(seq_idx), _ptr(pos), ctypes.byref(cache.c),

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -54,6 +55,15 @@ template <> struct Store<bf16> {
   static __device__ __forceinline__ float cvt(bf16 v) { return __bfloat162float(v); }
   static __device__ __forceinline__ void st(bf16* p, float v) { *p = __float2bfloat16_rn(v); }
   static __device__ __forceinline__ void st64(bf16* p, double v) { *p = __double2bfloat16(v); }
+};
+
+// E4M3 codes of the FP8 cache (the scale of the row is applied by the reader).
+template <> struct Store<__nv_fp8_e4m3> {
+  static __device__ __forceinline__ float ld(const __nv_fp8_e4m3* p) { return static_cast<float>(*p); }
+  // nearest E4M3, ties to even, straight from the double; saturating at +-448
+  static __device__ __forceinline__ void st64(__nv_fp8_e4m3* p, double v) {
+    p->__x = __nv_cvt_double_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+  }
 };
 
 template <typename T> __device__ __forceinline__ double to_f64(T v);

@@ -825,7 +825,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 // ================================================================ host side
 inline bool supports(const mla_config* c) {
-  return c->dtype == MLA_BF16 && c->n_heads == kH && c->d_c == kDc && c->d_r == kDr && c->block_size == kBS;
+  return c->dtype == MLA_BF16 && !(c->flags & MLA_FLAG_FP8_CACHE) && c->n_heads == kH && c->d_c == kDc &&
+         c->d_r == kDr && c->block_size == kBS;
 }
 
 // Bytes of packed query the decode keeps in its workspace per query row

@@ -1,5 +1,7 @@
 // Latent-space decode on CUDA cores: one warp per (segment, head).
-// Used for the fp32 storage path (small shapes, exact fp32 arithmetic).
+// Used for the fp32 storage path (small shapes, exact fp32 arithmetic) and
+// for the FP8 cache (E4M3 codes times the row's fp32 scale, `row_scale`
+// [num_blocks, block]; null for the other storage types).
 //
 // For the rows u of its segment (all visible to the segment's query row):
 //   s_u = (q_lat . c_u + q_R . kR_u) * scale * log2(e)
@@ -15,7 +17,7 @@ constexpr int kSimtDecodeMaxRow = 1024;  // d_c + d_r handled by one warp (32 la
 template <typename T, int DPL>
 __global__ void __launch_bounds__(128) decode_simt_kernel(
     const float* __restrict__ q_lat, const float* __restrict__ q_rope, const T* __restrict__ pool,
-    const int32_t* __restrict__ block_table, int max_blocks, int num_blocks,
+    const float* __restrict__ row_scale, const int32_t* __restrict__ block_table, int max_blocks, int num_blocks,
     const int32_t* __restrict__ seq_lens, int n_q, int H, int d_c, int d_r, int bs,
     float scale_log2, void* ws, DecodeLayout L) {
   const DecodeHeader* hd = ws_at<DecodeHeader>(ws, 0);
@@ -51,12 +53,13 @@ __global__ void __launch_bounds__(128) decode_simt_kernel(
     const T* base = pool + (long long)phys * bs * row;
     for (int r = 0; r < nrows; ++r) {
       const T* kv = base + (long long)r * row;
+      const float sc = row_scale != nullptr ? row_scale[(long long)phys * bs + r] : 1.f;
       float part = 0.f;
       float c[DPL];
 #pragma unroll
       for (int i = 0; i < DPL; ++i) {
         const int d = lane + 32 * i;
-        c[i] = d < row ? Store<T>::ld(kv + d) : 0.f;
+        c[i] = d < row ? Store<T>::ld(kv + d) * sc : 0.f;
         part = fmaf(q[i], c[i], part);
       }
       const float s = warp_sum(part) * scale_log2;

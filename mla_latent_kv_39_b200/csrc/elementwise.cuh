@@ -87,6 +87,52 @@ __global__ void append_finish_kernel(const double* __restrict__ C, int splits, i
   }
 }
 
+// The same epilogue into an FP8 cache: one CTA per new token assembles its
+// exact row [c | RoPE(k_R)] in fp64 (shared memory), takes the row's largest
+// magnitude m, the scale s = fp32(m / 448) (1 if that is 0) and writes the
+// E4M3 codes of row / s (nearest, ties to even, saturating) and s.
+__global__ void __launch_bounds__(256) append_finish_fp8_kernel(
+    const double* __restrict__ C, int n_tok, int d_c, int d_r, double theta, const int32_t* __restrict__ seq_idx,
+    const int32_t* __restrict__ pos, __nv_fp8_e4m3* __restrict__ pool, float* __restrict__ row_scale,
+    const int32_t* __restrict__ block_table, int batch, int max_blocks, int num_blocks, int bs) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ double v[];  // [d_c + d_r]
+  __shared__ double warp_max[8];
+  __shared__ long long slot_s;
+  const int t = blockIdx.x, row = d_c + d_r;
+  if (t >= n_tok) return;
+  if (threadIdx.x == 0) slot_s = cache_row_slot(seq_idx, pos, t, block_table, batch, max_blocks, num_blocks, bs);
+  const double* src = C + (long long)t * row;
+  for (int k = threadIdx.x; k < d_c + d_r / 2; k += blockDim.x) {
+    if (k < d_c) {
+      v[k] = src[k];
+    } else {
+      const int pr = k - d_c;  // rotary pair index
+      double sn, cs;
+      sincos((double)pos[t] * rope_inv_freq(theta, pr, d_r), &sn, &cs);
+      const double r0 = src[d_c + 2 * pr], r1 = src[d_c + 2 * pr + 1];
+      v[d_c + 2 * pr] = r0 * cs - r1 * sn;
+      v[d_c + 2 * pr + 1] = r0 * sn + r1 * cs;
+    }
+  }
+  __syncthreads();
+  double m = 0.0;
+  for (int k = threadIdx.x; k < row; k += blockDim.x) m = fmax(m, fabs(v[k]));
+  for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  const long long slot = slot_s;
+  if (slot < 0) return;
+  m = 0.0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmax(m, warp_max[w]);
+  float scale = __double2float_rn(m / 448.0);
+  if (scale == 0.f) scale = 1.f;
+  __nv_fp8_e4m3* dst = pool + slot * row;
+  for (int k = threadIdx.x; k < row; k += blockDim.x) Store<__nv_fp8_e4m3>::st64(dst + k, v[k] / (double)scale);
+  if (threadIdx.x == 0) row_scale[slot] = scale;
+}
+
 // Split q [n, H, nope + d_r] (fp32) into q_nope (storage type) and the rotated
 // q_rope (storage type).  The RoPE angle and rotation are evaluated in fp64.
 template <typename T>

@@ -28,13 +28,27 @@ mla_status check_cfg(const mla_config* c) {
       !(c->rope_theta > 0.0) || c->softmax_scale < 0.f)
     return MLA_ERR_INVALID_ARG;
   if (c->dtype != MLA_F32 && c->dtype != MLA_BF16) return MLA_ERR_INVALID_ARG;
-  if (c->flags & ~MLA_FLAG_SPLIT_QUERY) return MLA_ERR_INVALID_ARG;
+  if (c->flags & ~(MLA_FLAG_SPLIT_QUERY | MLA_FLAG_FP8_CACHE)) return MLA_ERR_INVALID_ARG;
+  if ((c->flags & MLA_FLAG_FP8_CACHE) && c->dtype != MLA_BF16) return MLA_ERR_INVALID_ARG;
   return MLA_OK;
 }
+
+inline bool fp8_cache(const mla_config* c) { return (c->flags & MLA_FLAG_FP8_CACHE) != 0; }
+
+// The bf16 tensor-core decode (pair kernel, packed query): bf16 pages only.
+inline bool tc_decode(const mla_config* c) { return c->dtype == MLA_BF16 && !fp8_cache(c); }
 
 mla_status check_cache(const mla_cache* k) {
   if (!k || !k->pool || !k->block_table || k->num_blocks <= 0 || k->batch <= 0 ||
       k->max_blocks_per_seq <= 0)
+    return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+
+mla_status check_cache(const mla_config* c, const mla_cache* k) {
+  const mla_status st0 = check_cache(k);
+  if (st0 != MLA_OK) return st0;
+  if (fp8_cache(c) && (k->row_scale == nullptr || (reinterpret_cast<uintptr_t>(k->row_scale) & 3u)))
     return MLA_ERR_INVALID_ARG;
   return MLA_OK;
 }
@@ -101,6 +115,13 @@ mla_status append_impl(const mla_config* c, const void* x, int n, const void* W_
     GemmSimtArgs g2{x, W_KR, C + c->d_c, n, c->d_r, Kc, S, c->hidden, 1, Kc, c->d_r, 1, (long long)Kc * c->d_r,
                     row, 1, 0};
     MLA_CUDA((gemm_simt<T, T, double, true>(g2, s)));
+  }
+  if (c->flags & MLA_FLAG_FP8_CACHE) {
+    const size_t smem = sizeof(double) * (size_t)row;
+    if (smem > 48 * 1024) return MLA_ERR_UNSUPPORTED;
+    return st(launch_chained(append_finish_fp8_kernel, dim3(n), dim3(256), smem, s, (const double*)C, n, c->d_c,
+                             c->d_r, c->rope_theta, seq_idx, pos, static_cast<__nv_fp8_e4m3*>(k->pool), k->row_scale,
+                             k->block_table, k->batch, k->max_blocks_per_seq, k->num_blocks, c->block_size));
   }
   const long long total = (long long)n * (c->d_c + c->d_r / 2);
   return st(launch_chained(append_finish_kernel<T>, dim3(grid_for(total)), dim3(256), 0, s, (const double*)C, 1, n,
@@ -324,19 +345,19 @@ mla_status out_tc(const mla_config* c, const float* o_lat, int n, const void* W_
 // tensor-core path (bf16), two warps-worth of CTAs per SM on the CUDA-core path.
 int default_workers(const mla_config* c) {
   const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
-  if (c->dtype == MLA_BF16) return std::max(1, sms / 2);
+  if (tc_decode(c)) return std::max(1, sms / 2);
   return std::max(1, 2 * sms);
 }
 
 // The tensor-core decode reads the query as bf16 rows [H, d_c + d_r] that a
 // first kernel packs from the fp32 inputs into the workspace.
 size_t qpack_row_bytes(const mla_config* c) {
-  return c->dtype == MLA_BF16 ? pairdec::qpack_row_bytes(c) : 0;
+  return tc_decode(c) ? pairdec::qpack_row_bytes(c) : 0;
 }
 
 // Partial outputs of the split decode: bf16 from the tensor-core decode
 // (they feed bf16 MMAs next), fp32 from the CUDA-core one.
-int part_elem(const mla_config* c) { return c->dtype == MLA_BF16 ? 2 : 4; }
+int part_elem(const mla_config* c) { return tc_decode(c) ? 2 : 4; }
 
 
 int resolve_workers(const mla_config* c, int max_workers) {
@@ -350,7 +371,7 @@ void launch_decode_simt(const mla_config* c, const float* q_lat, const float* q_
   const float scale_log2 = scale_of(c) * 1.4426950408889634f;
   dim3 grid(L.max_segments, (c->n_heads + 3) / 4);
   decode_simt_kernel<T, DPL><<<grid, 128, 0, s>>>(
-      q_lat, q_rope, static_cast<const T*>(k->pool),
+      q_lat, q_rope, static_cast<const T*>(k->pool), fp8_cache(c) ? k->row_scale : nullptr,
       k->block_table, k->max_blocks_per_seq, k->num_blocks, seq_lens, n_q, c->n_heads, c->d_c, c->d_r,
       c->block_size, scale_log2, ws, L);
   note_launch();
@@ -465,7 +486,7 @@ mla_status mla_cache_append(const mla_config* cfg, const void* x, int32_t n_tok,
   if (n_tok < 0) return MLA_ERR_INVALID_ARG;
   if (n_tok == 0) return MLA_OK;
   if (!x || !W_DKV || !W_KR || !seq_idx || !pos || !workspace) return MLA_ERR_INVALID_ARG;
-  MLA_TRY(check_cache(cache));
+  MLA_TRY(check_cache(cfg, cache));
   if (ws_bytes < append_ws(cfg, n_tok)) return MLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cfg->dtype == MLA_BF16)
@@ -480,7 +501,7 @@ mla_status mla_cache_append_noalloc(const mla_config* cfg, const void* x, int32_
   if (n_tok < 0) return MLA_ERR_INVALID_ARG;
   if (n_tok == 0) return MLA_OK;
   if (!x || !W_DKV || !W_KR || !seq_idx || !pos) return MLA_ERR_INVALID_ARG;
-  MLA_TRY(check_cache(cache));
+  MLA_TRY(check_cache(cfg, cache));
   const size_t need = append_ws(cfg, n_tok);
   if (need > (size_t)MLA_APPEND_NOALLOC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
   void* scratch = nullptr;
@@ -519,7 +540,7 @@ mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok, con
 }
 
 size_t mla_query_packed_bytes(const mla_config* cfg, int32_t n_tok) {
-  if (check_cfg(cfg) != MLA_OK || n_tok < 0 || cfg->dtype != MLA_BF16) return 0;
+  if (check_cfg(cfg) != MLA_OK || n_tok < 0 || !tc_decode(cfg)) return 0;
   return (size_t)n_tok * pairdec::qpack_row_bytes(cfg);
 }
 
@@ -546,7 +567,7 @@ static mla_status decode_packed_impl(const mla_config* cfg, const void* q_packed
   if (batch == 0) return MLA_OK;
   if (!q_packed || !seq_lens || !workspace) return MLA_ERR_INVALID_ARG;
   if ((long long)batch * n_q > kPlanMaxRows) return MLA_ERR_UNSUPPORTED;
-  MLA_TRY(check_cache(cache));
+  MLA_TRY(check_cache(cfg, cache));
   if (cache->batch < batch) return MLA_ERR_INVALID_ARG;
   if (cfg->dtype != MLA_BF16 || !pairdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
   if (!all_aligned16(q_packed, cache->pool, workspace)) return MLA_ERR_INVALID_ARG;
@@ -580,7 +601,7 @@ mla_status mla_decode_plan(const mla_config* cfg, int32_t batch, int32_t n_q, co
   if (batch == 0) return MLA_OK;
   if (!seq_lens || !workspace) return MLA_ERR_INVALID_ARG;
   if ((long long)batch * n_q > kPlanMaxRows) return MLA_ERR_UNSUPPORTED;
-  MLA_TRY(check_cache(cache));
+  MLA_TRY(check_cache(cfg, cache));
   if (cache->batch < batch) return MLA_ERR_INVALID_ARG;
   if (!all_aligned16(workspace)) return MLA_ERR_INVALID_ARG;
   const DecodeLayout L = decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers),
@@ -610,16 +631,16 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
   if (batch == 0) return MLA_OK;
   if (!q_lat || !q_rope || !seq_lens || !workspace) return MLA_ERR_INVALID_ARG;
   if ((long long)batch * n_q > kPlanMaxRows) return MLA_ERR_UNSUPPORTED;
-  MLA_TRY(check_cache(cache));
+  MLA_TRY(check_cache(cfg, cache));
   if (cache->batch < batch) return MLA_ERR_INVALID_ARG;
-  if (cfg->dtype == MLA_BF16 && !pairdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
-  if (cfg->dtype == MLA_BF16 && !all_aligned16(q_lat, q_rope, cache->pool, workspace)) return MLA_ERR_INVALID_ARG;
+  if (tc_decode(cfg) && !pairdec::supports(cfg)) return MLA_ERR_UNSUPPORTED;
+  if (tc_decode(cfg) && !all_aligned16(q_lat, q_rope, cache->pool, workspace)) return MLA_ERR_INVALID_ARG;
   const DecodeLayout L =
       decode_layout(batch, n_q, cfg->n_heads, cfg->d_c, resolve_workers(cfg, max_workers), qpack_row_bytes(cfg),
                     part_elem(cfg));
   if (ws_bytes < (size_t)L.total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cfg->dtype == MLA_BF16)
+  if (tc_decode(cfg))
     return pairdec::launch(cfg, q_lat, q_rope, nullptr, n_q, cache, seq_lens, workspace, L, scale_of(cfg),
                            g_wait_limit_ns.load(std::memory_order_relaxed), s);
   const size_t plan_smem = sizeof(int) * ((size_t)batch * n_q + 1);
@@ -629,6 +650,8 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
     return MLA_ERR_CUDA;
   MLA_CUDA(launch_chained(decode_plan_kernel, dim3(1), dim3(1024), plan_smem, s, seq_lens, cfg->block_size,
                           cache->max_blocks_per_seq, workspace, L));
+  if (fp8_cache(cfg))
+    return decode_simt_dispatch<__nv_fp8_e4m3>(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, s);
   return decode_simt_dispatch<float>(cfg, q_lat, q_rope, n_q, cache, seq_lens, workspace, L, s);
 }
 

@@ -16,5 +16,6 @@ from .workloads import (  # noqa: F401
     generate,
     reduced,
     build_pool,
+    build_row_scale,
     device_inputs,
 )

@@ -18,7 +18,12 @@ with ``workload.seed`` (fixed so that every consumer sees identical values):
    ``[sum L_b, d_c + d_r]`` drawn N(0, 1) directly, optionally with a
    Bernoulli(frac) subset of rows scaled by ``spike_scale``;
 5. the physical block permutation of the paged pool (``randperm``), when
-   the workload asks for shuffled blocks.
+   the workload asks for shuffled blocks;
+6. for an FP8 cache (``fp8_cache``), instead of step 4's latent rows: E4M3
+   codes ``[sum L_b, d_c + d_r]`` (sign, exponent field in 6..15 and
+   mantissa field uniform, never the NaN pattern: magnitudes 2^-1 .. 448)
+   and one fp32 scale per row, ``0.002 + 0.01 |N(0, 1)|``.  They are drawn
+   after step 5, as codes are stored bytes, not values.
 """
 
 from __future__ import annotations
@@ -114,6 +119,13 @@ class Workload:
     # run option, not data: hold the query as a bf16 hi + lo pair in the decode
     # (strongly peaked softmaxes need more than bf16's 8 significant bits)
     split_query: bool = False
+    # the cache holds E4M3 codes and one fp32 scale per row (weights stay bf16)
+    fp8_cache: bool = False
+
+    @property
+    def cache_row_bytes(self) -> int:
+        """Bytes of one cached row (with its scale for an FP8 cache)."""
+        return self.shape.row + 4 if self.fp8_cache else self.shape.row * self.shape.elem_bytes
 
     @property
     def n_tok(self) -> int:
@@ -138,6 +150,11 @@ WORKLOADS: Dict[str, Workload] = {
         spike_frac=0.01, spike_scale=8.0, split_query=True,
         description="V3-shaped long-context split-KV stress, contexts 65536/131072/32768/100000, "
                     "1% of latent rows scaled x8"),
+    "v3_fp8_b64_ragged1k_8k": Workload(
+        "v3_fp8_b64_ragged1k_8k", SHAPES["v3"], batch=64, n_q=1, len_lo=1024, len_hi=8192,
+        shuffled_blocks=True, fp8_cache=True,
+        description="the batch-64 V3 decode over an FP8 latent cache (E4M3 codes + fp32 row scale), "
+                    "ragged lengths U[1024, 8192], 64-token pages in shuffled order"),
     "v3_b128_nq2_ragged512_16k": Workload(
         "v3_b128_nq2_ragged512_16k", SHAPES["v3"], batch=128, n_q=2, len_lo=512, len_hi=16384,
         description="V3-shaped multi-token decode, batch 128, 2 causal query tokens per sequence, "
@@ -186,12 +203,14 @@ class WorkloadData:
     weights: Dict[str, torch.Tensor]
     cached_len: torch.Tensor              # int64 [B]: rows already in the cache
     x_new: torch.Tensor                   # [B*n_q, hidden], row b*n_q + j is token j of seq b
-    cached_rows: Optional[torch.Tensor]   # [sum L_b, d_c + d_r] latent rows (None if from append)
+    cached_rows: Optional[torch.Tensor]   # [sum L_b, d_c + d_r] latent rows (None if from append or FP8)
     x_cached: Optional[torch.Tensor]      # [sum L_b, hidden] (only when cached_from_append)
     spike_mask: Optional[torch.Tensor]    # bool [sum L_b] rows scaled by spike_scale
     block_table: torch.Tensor             # int32 [B, max_blocks]
     num_blocks: int
     row_offsets: torch.Tensor = field(default=None)  # int64 [B+1] start of seq b in cached rows
+    cached_codes: Optional[torch.Tensor] = None      # uint8 [sum L_b, d_c + d_r] E4M3 codes (FP8 cache)
+    cached_scale: Optional[torch.Tensor] = None      # float32 [sum L_b] their row scales
 
     @property
     def seq_lens(self) -> torch.Tensor:
@@ -264,6 +283,8 @@ def generate(wl: Workload, *, with_weights: bool = True) -> WorkloadData:
     cached_rows = x_cached = spike_mask = None
     if wl.cached_from_append:
         x_cached = torch.randn(total, shape.hidden, generator=g, dtype=torch.float32).to(dt)
+    elif wl.fp8_cache:
+        pass  # codes and scales after the block table (step 6)
     else:
         cached_rows = _draw_rows(total, shape.row, dt, g)
         if wl.spike_frac > 0.0:
@@ -287,8 +308,17 @@ def generate(wl: Workload, *, with_weights: bool = True) -> WorkloadData:
         block_table[b, :nb] = physical[start:start + nb].to(torch.int32)
         start += nb
 
+    codes = scales = None
+    if wl.fp8_cache and not wl.cached_from_append:
+        sign = torch.randint(0, 2, (total, shape.row), generator=g, dtype=torch.int32)
+        expo = torch.randint(6, 16, (total, shape.row), generator=g, dtype=torch.int32)
+        mant = torch.randint(0, 8, (total, shape.row), generator=g, dtype=torch.int32)
+        mant = torch.where((expo == 15) & (mant == 7), torch.full_like(mant, 6), mant)   # 0x7F / 0xFF: NaN
+        codes = ((sign << 7) | (expo << 3) | mant).to(torch.uint8)
+        scales = (0.002 + 0.01 * torch.randn(total, generator=g).abs()).to(torch.float32)
+
     return WorkloadData(wl, weights, cached_len, x_new, cached_rows, x_cached, spike_mask,
-                        block_table, num_blocks, row_offsets)
+                        block_table, num_blocks, row_offsets, codes, scales)
 
 
 def build_pool(data: WorkloadData, rows: Optional[torch.Tensor] = None,
@@ -303,9 +333,20 @@ def build_pool(data: WorkloadData, rows: Optional[torch.Tensor] = None,
     wl = data.workload
     shape = wl.shape
     bs = shape.block_size
+    if wl.fp8_cache:   # E4M3 codes; unwritten slots hold the NaN code 0x7F
+        src = data.cached_codes if rows is None else rows
+        pool = torch.full((max(data.num_blocks, 1), bs, shape.row), 0x7F, dtype=torch.uint8)
+        return _scatter(data, pool, src)
     src = data.cached_rows if rows is None else rows
     pool = torch.full((max(data.num_blocks, 1), bs, shape.row), fill, dtype=shape.torch_dtype)
-    flat = pool.view(-1, shape.row)
+    return _scatter(data, pool, src)
+
+
+def _scatter(data: WorkloadData, pool: torch.Tensor, src: Optional[torch.Tensor]) -> torch.Tensor:
+    """Row ``t`` of sequence ``b`` of ``src`` -> ``pool[block_table[b, t // block], t % block]``."""
+    wl = data.workload
+    bs = wl.shape.block_size
+    flat = pool.view(pool.shape[0] * pool.shape[1], *pool.shape[2:])
     if src is None:          # rows are produced later by the append step
         return pool
     for b in range(wl.batch):
@@ -320,6 +361,16 @@ def build_pool(data: WorkloadData, rows: Optional[torch.Tensor] = None,
     return pool
 
 
+def build_row_scale(data: WorkloadData) -> Optional[torch.Tensor]:
+    """FP8 cache: the rows' scales in the pool's layout ``[num_blocks, block]``
+    (unwritten slots NaN); None for other caches."""
+    if not data.workload.fp8_cache:
+        return None
+    bs = data.workload.shape.block_size
+    scale = torch.full((max(data.num_blocks, 1), bs), float("nan"), dtype=torch.float32)
+    return _scatter(data, scale, data.cached_scale)
+
+
 def device_inputs(data: WorkloadData, device, pool: Optional[torch.Tensor] = None) -> Dict[str, object]:
     """Copies of the seeded inputs on ``device`` (pure data movement)."""
     dev = torch.device(device)
@@ -331,6 +382,7 @@ def device_inputs(data: WorkloadData, device, pool: Optional[torch.Tensor] = Non
         "x_new": data.x_new.to(dev),
         "pos": data.new_positions().to(dev),
         "seq_idx": data.new_seq_idx().to(dev),
+        "row_scale": None if not data.workload.fp8_cache else build_row_scale(data).to(dev),
     }
     if data.x_cached is not None:
         L = int(data.cached_len.sum())

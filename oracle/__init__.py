@@ -20,6 +20,12 @@ Parity status per function (pins live in ``tests/test_oracle_pins.py``):
 * ``heads_from_latent`` and
   ``output_projection``       pinned (through the order-swap check and brute force)
 * cache-size formulas         pinned (every byte count the pages print)
+* ``e4m3_value``              pinned (every one of the 256 codes against torch's
+                              float8_e4m3fn)
+* ``round_to_e4m3``           pinned (torch's fp32 -> float8_e4m3fn cast on fp32
+                              values within +-448, ties, subnormals, saturation)
+* ``fp8_row_quantize``        pinned (the largest magnitude maps to 448, every value
+                              within half a code step, zero rows)
 """
 
 from .mla import (  # noqa: F401
@@ -28,6 +34,11 @@ from .mla import (  # noqa: F401
     rope,
     softmax_scale,
     latent_rows,
+    latent_rows_exact,
+    e4m3_value,
+    e4m3_code,
+    round_to_e4m3,
+    fp8_row_quantize,
     queries,
     absorb_query,
     attend_decompressed,

@@ -75,6 +75,69 @@ def round_to_storage(a, dtype: str) -> np.ndarray:
     raise ValueError(f"unknown storage dtype {dtype!r}")
 
 
+# OCP 8-bit floating point, E4M3 variant: 1 sign bit, 4 exponent bits (bias
+# 7), 3 mantissa bits; no infinities, exponent field 15 with mantissa 7 is
+# NaN, so the largest finite magnitude is 1.75 * 2**8 = 448; subnormals
+# (exponent field 0) are m * 2**-9.  The pages fix no cache number format;
+# this is the common FP8 cache format, with one scale per row ("MLA ve diğer
+# optimizasyonlarla ilişkisi": quantization is used together with MLA).
+_E4M3_MAX = 448.0
+
+
+def e4m3_value(codes) -> np.ndarray:
+    """The value of each E4M3 byte (uint8 array), as float64 (NaN codes -> NaN)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.power(2.0, e - 7))
+    mag = np.where((e == 15) & ((c & 0x7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def round_to_e4m3(a) -> np.ndarray:
+    """Nearest E4M3 value of each float64 entry, ties to even, magnitudes
+    beyond 448 saturating to +-448; as float64."""
+    a = np.asarray(a, dtype=np.float64)
+    out = np.array(a, dtype=np.float64, copy=True)
+    fin = np.isfinite(a) & (a != 0.0)
+    if np.any(fin):
+        v = a[fin]
+        _, e = np.frexp(v)                   # v = m * 2**e with 0.5 <= |m| < 1
+        q = np.maximum(e - 4, -9)            # 4 significant bits; subnormal step 2**-9
+        w = np.ldexp(np.rint(np.ldexp(v, -q)), q)
+        out[fin] = np.clip(w, -_E4M3_MAX, _E4M3_MAX)
+    return out
+
+
+def e4m3_code(values) -> np.ndarray:
+    """The byte of each E4M3 value (inverse of ``e4m3_value`` on finite
+    values; the sign of a zero is kept: -0 is 0x80)."""
+    v = np.asarray(values, dtype=np.float64)
+    table = e4m3_value(np.arange(256, dtype=np.uint8))
+    codes = np.zeros(v.shape, dtype=np.uint8)
+    for c in range(256):
+        if table[c] == 0.0 or not np.isfinite(table[c]):
+            continue
+        codes[v == table[c]] = c
+    codes[(v == 0.0) & np.signbit(v)] = 0x80
+    return codes
+
+
+def fp8_row_quantize(rows) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-row scaled E4M3 of float64 rows ``[..., width]``.
+
+    ``scale = fp32(max |row| / 448)`` (1 where that is 0); the stored codes
+    are ``round_to_e4m3(row / scale)``.  Returns ``(code_values, scale)`` as
+    float64; the cached row stands for ``code_values * scale``.
+    """
+    r = np.asarray(rows, dtype=np.float64)
+    amax = np.max(np.abs(r), axis=-1)
+    scale = (amax / _E4M3_MAX).astype(np.float32).astype(np.float64)
+    scale = np.where(scale == 0.0, 1.0, scale)
+    return round_to_e4m3(r / scale[..., None]), scale
+
+
 def to64(t) -> np.ndarray:
     """A CPU tensor or array as float64 NumPy (bf16 and fp32 widen exactly)."""
     if hasattr(t, "detach"):
@@ -118,16 +181,24 @@ def softmax_scale(qk_nope: int, d_r: int) -> float:
 # Step 1: hidden -> latent row (the cache)
 # --------------------------------------------------------------------------
 
-def latent_rows(x, W_DKV, W_KR, pos, theta: float, dtype: str) -> Tuple[np.ndarray, np.ndarray]:
-    """Cache rows ``(c_KV, k_R)`` of tokens ``x`` at absolute positions ``pos``.
-
-    ``c_KV = x W_DKV`` (the compressed latent) and ``k_R = RoPE(x W_KR, pos)``
-    (the decoupled rotary key), each rounded once to the cache storage type.
-    """
+def latent_rows_exact(x, W_DKV, W_KR, pos, theta: float) -> Tuple[np.ndarray, np.ndarray]:
+    """``c_KV = x W_DKV`` (the compressed latent) and ``k_R = RoPE(x W_KR, pos)``
+    (the decoupled rotary key) of tokens ``x`` at positions ``pos``, unrounded."""
     x = to64(x)
     c = x @ to64(W_DKV)
     r = x @ to64(W_KR)
-    k_r = rope(r, np.asarray(pos), theta)
+    return c, rope(r, np.asarray(pos), theta)
+
+
+def latent_rows(x, W_DKV, W_KR, pos, theta: float, dtype: str) -> Tuple[np.ndarray, np.ndarray]:
+    """Cache rows ``(c_KV, k_R)`` of tokens ``x`` at absolute positions ``pos``,
+    each value rounded once to the cache storage type; for ``"fp8"`` the
+    values the FP8 rows stand for (``fp8_row_quantize`` of ``[c_KV | k_R]``)."""
+    c, k_r = latent_rows_exact(x, W_DKV, W_KR, pos, theta)
+    if dtype == "fp8":
+        codes, scale = fp8_row_quantize(np.concatenate([c, k_r], axis=-1))
+        v = codes * scale[..., None]
+        return v[..., :c.shape[-1]], v[..., c.shape[-1]:]
     return round_to_storage(c, dtype), round_to_storage(k_r, dtype)
 
 
@@ -262,7 +333,7 @@ def output_projection(o_heads, W_O) -> np.ndarray:
 
 def decode_step(shape, weights, x_new, pos_new, cached_c: Sequence, cached_kr: Sequence,
                 n_q: int, order: str = "decompressed", seqs: Optional[Iterable[int]] = None,
-                want_y: bool = True) -> Dict[str, object]:
+                want_y: bool = True, cache_dtype: Optional[str] = None) -> Dict[str, object]:
     """One decode step of one layer (cache append, queries, attention, output).
 
     ``cached_c[b]`` / ``cached_kr[b]`` are the rows already cached for
@@ -276,13 +347,15 @@ def decode_step(shape, weights, x_new, pos_new, cached_c: Sequence, cached_kr: S
     Returns a dict with ``c_new, kr_new, q_nope, q_r, q_lat`` for every token
     and, per attended token t (dict keyed by t), ``o_heads`` and, in the
     absorbed order, ``o_lat``/``lse``; plus ``y`` rows for attended tokens.
+    ``cache_dtype`` ("fp8" for the E4M3 cache) overrides the storage type of
+    the appended rows, which is otherwise the shape's.
     """
     H, nope, dr, dv = shape.n_heads, shape.qk_nope, shape.d_r, shape.v_head
     scale = softmax_scale(nope, dr)
     W = {k: to64(v) for k, v in weights.items()}
     pos_new = np.asarray(pos_new)
     c_new, kr_new = latent_rows(x_new, W["W_DKV"], W["W_KR"], pos_new, shape.rope_theta,
-                                shape.dtype)
+                                cache_dtype or shape.dtype)
     q_nope, q_r = queries(x_new, W, H, nope, dr, pos_new, shape.rope_theta)
     q_lat = absorb_query(q_nope, W["W_UK"], H, nope)
     B = len(cached_c)

@@ -21,8 +21,8 @@ def tol_for(shape) -> float:
 def run_gpu(wl, data=None, max_workers: int = 0, pool: Optional[torch.Tensor] = None, packed_query: bool = True):
     data = data if data is not None else generate(wl)
     dev = device_inputs(data, "cuda", pool=pool)
-    cfg = Config.from_shape(wl.shape, split_query=wl.split_query)
-    cache = Cache(dev["pool"], dev["block_table"])
+    cfg = Config.from_shape(wl.shape, split_query=wl.split_query, fp8_cache=wl.fp8_cache)
+    cache = Cache(dev["pool"], dev["block_table"], dev["row_scale"])
     layer = DecodeLayer(cfg, dev["weights"], cache, wl.batch, wl.n_q, max_workers, packed_query=packed_query)
     if wl.cached_from_append:
         layer.append(dev["x_cached"], dev["seq_idx_cached"], dev["pos_cached"])
@@ -41,6 +41,10 @@ def oracle_cached_rows(data):
         if wl.cached_from_append:
             c, kr = oracle.latent_rows(data.x_cached[s:e], data.weights["W_DKV"], data.weights["W_KR"],
                                        np.arange(e - s), shape.rope_theta, shape.dtype)
+        elif wl.fp8_cache:     # the values the stored codes and scales stand for
+            rows = oracle.e4m3_value(data.cached_codes[s:e].numpy()) * \
+                oracle.to64(data.cached_scale[s:e])[:, None]
+            c, kr = rows[:, :shape.d_c], rows[:, shape.d_c:]
         else:
             rows = oracle.to64(data.cached_rows[s:e])
             c, kr = rows[:, :shape.d_c], rows[:, shape.d_c:]
@@ -53,7 +57,7 @@ def oracle_expect(data, seqs: Optional[Iterable[int]] = None, order: str = "abso
     wl = data.workload
     cc, ck = oracle_cached_rows(data)
     out = oracle.decode_step(wl.shape, data.weights, data.x_new, data.new_positions().numpy(), cc, ck,
-                             wl.n_q, order=order, seqs=seqs)
+                             wl.n_q, order=order, seqs=seqs, cache_dtype="fp8" if wl.fp8_cache else None)
     out["cached_c"], out["cached_kr"] = cc, ck
     return out
 
@@ -76,9 +80,25 @@ def pool_row(layer, data, b: int, p: int) -> np.ndarray:
 
 
 def check_new_cache_rows(layer, data, exp):
-    """Rows appended by the step are bit-identical to the oracle's rounded rows."""
+    """Rows appended by the step are bit-identical to the oracle's rounded rows
+    (for an FP8 cache: the E4M3 bytes and the fp32 row scale)."""
     wl = data.workload
     pos = data.new_positions().numpy()
+    if wl.fp8_cache:
+        W = data.weights
+        c, k = oracle.latent_rows_exact(data.x_new, W["W_DKV"], W["W_KR"], pos, wl.shape.rope_theta)
+        codes, scale = oracle.fp8_row_quantize(np.concatenate([c, k], axis=1))
+        want = oracle.e4m3_code(codes)
+        bs = wl.shape.block_size
+        for t in range(wl.n_tok):
+            b = t // wl.n_q
+            page = int(data.block_table[b, int(pos[t]) // bs])
+            got = layer.cache.pool[page, int(pos[t]) % bs].cpu().numpy()
+            bad = np.nonzero(got != want[t])[0]
+            assert bad.size == 0, f"token {t}: {bad.size} FP8 codes differ, first at {bad[:5]}"
+            got_s = float(layer.cache.row_scale[page, int(pos[t]) % bs].cpu())
+            assert got_s == scale[t], f"token {t}: row scale {got_s!r} != {scale[t]!r}"
+        return
     want = np.concatenate([exp["c_new"], exp["kr_new"]], axis=1)
     for t in range(wl.n_tok):
         b = t // wl.n_q

@@ -45,16 +45,17 @@ def test_struct_layout_matches_the_header(tmp_path):
     src = tmp_path / "layout.c"
     src.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "mla.h"\n'
-        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu\\n\", sizeof(mla_config),"
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(mla_config),"
         " offsetof(mla_config, rope_theta), offsetof(mla_config, flags), sizeof(mla_cache),"
-        " offsetof(mla_cache, block_table), offsetof(mla_cache, max_blocks_per_seq));return 0;}\n")
+        " offsetof(mla_cache, block_table), offsetof(mla_cache, max_blocks_per_seq),"
+        " offsetof(mla_cache, row_scale));return 0;}\n")
     exe = tmp_path / "layout"
     subprocess.run(["gcc", f"-I{ROOT / 'include'}", str(src), "-o", str(exe)], check=True)
     got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True,
                                           check=True).stdout.split()]
     want = [ctypes.sizeof(abi.MLAConfig), abi.MLAConfig.rope_theta.offset, abi.MLAConfig.flags.offset,
             ctypes.sizeof(abi.MLACache), abi.MLACache.block_table.offset,
-            abi.MLACache.max_blocks_per_seq.offset]
+            abi.MLACache.max_blocks_per_seq.offset, abi.MLACache.row_scale.offset]
     assert got == want
 
 
@@ -65,7 +66,7 @@ def _cfg(**kw):
 
 
 def test_abi_version(lib):
-    assert lib.mla_abi_version() == 1
+    assert lib.mla_abi_version() == 2
 
 
 def test_invalid_configs_are_rejected_synchronously(lib):

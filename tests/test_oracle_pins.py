@@ -403,3 +403,60 @@ def test_a_planted_dropped_rotary_term_is_caught(monkeypatch):
     monkeypatch.setattr(m, "attend_absorbed", wrong)
     with pytest.raises(AssertionError):
         test_oracle_matches_brute_force_loops(1, BRUTE_SHAPE)
+
+
+# ---------------------------------------------------------------- FP8 cache format
+
+def test_e4m3_value_of_every_code_matches_torch_float8_e4m3fn():
+    codes = np.arange(256, dtype=np.uint8)
+    mine = oracle.e4m3_value(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    assert np.array_equal(mine[~np.isnan(mine)], ref[~np.isnan(ref)])
+    assert np.nanmax(mine) == 448.0 and oracle.e4m3_value(np.array([1], np.uint8))[0] == 2.0 ** -9
+    assert np.isnan(mine[0x7F]) and np.isnan(mine[0xFF]) and np.sum(np.isnan(mine)) == 2
+
+
+def test_round_to_e4m3_matches_torch_on_fp32_values_and_ties():
+    g = np.random.default_rng(5)
+    x = (g.standard_normal(100000) * np.exp(g.uniform(-14, 6.5, 100000))).astype(np.float32)
+    x = x[np.abs(x) <= 448]
+    table = oracle.e4m3_value(np.arange(256, dtype=np.uint8))
+    grid = np.unique(table[np.isfinite(table)])
+    ties = ((grid[:-1] + grid[1:]) / 2).astype(np.float32)       # exact midpoints (fp32-exact)
+    for v in (x, ties):
+        ref = torch.from_numpy(v).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+        assert np.array_equal(oracle.round_to_e4m3(v.astype(np.float64)), ref)
+    # ties to even: 1 + 1/16 lies between 1 and 1.125 -> 1 (even mantissa); 1 + 3/16 -> 1.25
+    assert oracle.round_to_e4m3(np.array([1.0625, 1.1875, -1.0625]))[[0, 1, 2]].tolist() == [1.0, 1.25, -1.0]
+    # saturation beyond the largest finite value (torch gives NaN there)
+    assert oracle.round_to_e4m3(np.array([449.0, 1e9, -1e9])).tolist() == [448.0, 448.0, -448.0]
+    # one rounding from float64 (no fp32 detour): just above a tie goes up
+    above = 1.0625 + 2.0 ** -40
+    assert oracle.round_to_e4m3(np.array([above]))[0] == 1.125
+    codes = oracle.e4m3_code(np.array([1.0, -448.0, 2.0 ** -9, 0.0, -0.0]))
+    assert codes.tolist() == [0x38, 0xFE, 0x01, 0x00, 0x80]
+    every = np.arange(256, dtype=np.uint8)
+    finite = np.isfinite(oracle.e4m3_value(every))
+    assert np.array_equal(oracle.e4m3_code(oracle.e4m3_value(every))[finite], every[finite])
+    assert np.signbit(oracle.round_to_e4m3(np.array([-2.0 ** -12]))[0])    # underflow keeps the sign
+
+
+def test_fp8_row_quantize_maps_the_row_maximum_to_448_within_half_a_step():
+    g = np.random.default_rng(9)
+    rows = g.standard_normal((50, 576)) * np.exp(g.uniform(-8, 8, (50, 1)))
+    codes, scale = oracle.fp8_row_quantize(rows)
+    assert np.all(scale == scale.astype(np.float32).astype(np.float64))       # fp32 scales
+    assert np.all(np.max(np.abs(codes), axis=1) == 448.0)
+    # |row / s - code| <= half the code step at that magnitude (subnormal step 2^-9)
+    _, e = np.frexp(np.abs(codes) + (codes == 0))
+    step = np.ldexp(1.0, np.maximum(e - 4, -9))
+    assert np.all(np.abs(rows / scale[:, None] - codes) <= step / 2 * (1 + 1e-12))
+    # an all-zero row: scale 1, codes 0
+    z_codes, z_scale = oracle.fp8_row_quantize(np.zeros((1, 8)))
+    assert z_scale[0] == 1.0 and not np.any(z_codes)
+    # the fp8 storage path of latent_rows returns code * scale per row
+    c, k = oracle.latent_rows(rows[:3, :64], np.eye(64)[:, :48], np.eye(64)[:, 48:], np.zeros(3), 1e4, "fp8")
+    joined = np.concatenate([c, k], axis=1)
+    cc, ss = oracle.fp8_row_quantize(rows[:3, :64])
+    assert np.array_equal(joined, cc * ss[:, None])
