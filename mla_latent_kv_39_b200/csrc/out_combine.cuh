@@ -32,6 +32,7 @@ constexpr int kABytes = 128 * 128;     // 128 features x 64 k (two 64 x 64 boxes
 constexpr int kRingBytes = 176 * 1024;
 constexpr int kMaxStages = 8;
 constexpr int kMaxN = 512;
+constexpr int kVHead = 128;           // output features per head (the MMA M)
 
 // B rows a stage holds: all N columns in one box, or two boxes of 256 rows.
 __host__ __device__ constexpr int b_rows(int N) { return N <= 256 ? N : 512; }
@@ -51,6 +52,8 @@ struct Smem {
 };
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory over the 227 KiB per-block limit");
+// the output tile of the most rows a launch takes (rows <= segments <= kMaxN) fits the ring
+static_assert(kMaxN * kVHead * 2 <= kRingBytes, "output staging larger than the ring");
 
 struct Params {
   const void* ws;   // decode workspace (plan, log2-sum-exp, partial outputs)
@@ -177,19 +180,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int* sfirst = ws_at<int>(p.ws, L.off_seq_first);
     const int* snseg = ws_at<int>(p.ws, L.off_seq_nseg);
     const float* lse = ws_at<float>(p.ws, L.off_lse);
-    // merge weights of this head, one segment per thread (the MMAs run meanwhile)
+    // This head's log2-sum-exps and each segment's row, in one coalesced pass
+    // (the MMAs run meanwhile) ...
     for (int s = tid; s < nseg; s += 128) {
-      const int v = segs[s].x;
-      const RowMerge rm(lse, sfirst[v], snseg[v], p.H, h);
-      sm.w[s] = rm.weight(lse[(long long)s * p.H + h]);
-      sm.row[s] = v;
+      sm.w[s] = lse[(long long)s * p.H + h];
+      sm.row[s] = segs[s].x;
     }
+    __syncwarp();
     named_sync(1, 128);
-    bf16* out_h = p.oh + (long long)h * p.v_head + f;
-    const long long rstride = (long long)p.H * p.v_head;
+    // ... then, one row per thread, its merge weights in place: the segments
+    // of a row are contiguous and ordered (the RowMerge arithmetic, in order)
+    for (int v = tid; v < rows; v += 128) {
+      const int first = valid ? sfirst[v] : 0, n = valid ? snseg[v] : 0;
+      float M = -INFINITY;
+      for (int k = 0; k < n; ++k) M = fmaxf(M, sm.w[first + k]);
+      float Z = 0.f;
+      if (M != -INFINITY)
+        for (int k = 0; k < n; ++k) Z += exp2f(sm.w[first + k] - M);
+      const float invZ = M != -INFINITY ? 1.f / Z : 0.f;
+      for (int k = 0; k < n; ++k) sm.w[first + k] = invZ > 0.f ? exp2f(sm.w[first + k] - M) * invZ : 0.f;
+    }
+    __syncwarp();
+    named_sync(1, 128);
     bool ok = valid && __all_sync(0xffffffffu, mbar_wait(&sm.acc_full, 0, 103));
     if (valid && !ok) set_abort(sm);
     tc_fence_after();
+    // Every load and MMA on the ring is over: it holds the head's output rows
+    // as a bf16 tile [rows][v_head] (rows without a segment stay zero).
+    bf16* stage = reinterpret_cast<bf16*>(sm.ring);
+    for (int v = 0; v < rows; ++v) stage[v * kVHead + f] = __float2bfloat16_rn(0.f);
     int cur = -1;
     float acc = 0.f;
     for (int c0 = 0; ok && c0 < nseg; c0 += 32) {
@@ -202,20 +221,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (s >= nseg) break;
         const int v = sm.row[s];
         if (v != cur) {
-          if (cur >= 0) out_h[cur * rstride] = __float2bfloat16_rn(acc);
+          if (cur >= 0) stage[cur * kVHead + f] = __float2bfloat16_rn(acc);
           cur = v;
           acc = 0.f;
         }
         const float w = sm.w[s];
-        if (w != 0.f) acc = fmaf(w, __uint_as_float(d[k]), acc);
+        if (w != 0.f) acc = fmaf(w, __uint_as_float(d[k]), acc);  // a zero weight: never-written partial
       }
     }
-    if (cur >= 0) out_h[cur * rstride] = __float2bfloat16_rn(acc);
-    // rows without a segment (no visible rows, or no plan) are zero
-    for (int v = 0; v < rows; ++v)
-      if (!valid || snseg[v] == 0) out_h[v * rstride] = __float2bfloat16_rn(0.f);
+    if (cur >= 0) stage[cur * kVHead + f] = __float2bfloat16_rn(acc);
+    __syncwarp();
+    named_sync(1, 128);
+    // the tile out with 16-byte stores: a row's 256 bytes from 16 neighbouring threads
+    const long long rstride = (long long)p.H * kVHead;
+    for (int i = tid; i < rows * (kVHead / 8); i += 128) {
+      const int v = i / (kVHead / 8), c = i % (kVHead / 8);
+      *reinterpret_cast<uint4*>(p.oh + v * rstride + (long long)h * kVHead + 8 * c) =
+          *reinterpret_cast<const uint4*>(stage + v * kVHead + 8 * c);
+    }
   }
 
+  // The role branches above leave lanes of warps 0 and 1 apart (only lane 0
+  // runs the producer or issuer loop): reconverge each warp before the
+  // block-wide barrier, which counts whole warps.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -227,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ================================================================ host side
 inline bool supports(const mla_config* c, int max_segments) {
-  return c->dtype == MLA_BF16 && c->v_head == 128 && c->d_c % 64 == 0 && max_segments <= kMaxN;
+  return c->dtype == MLA_BF16 && c->v_head == kVHead && c->d_c % 64 == 0 && max_segments <= kMaxN;
 }
 
 inline mla_status make_maps(const void* W_UV, const void* ws, const DecodeLayout& L, const mla_config* c, int N,

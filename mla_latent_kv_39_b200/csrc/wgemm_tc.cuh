@@ -263,6 +263,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // The role branches above leave lanes of warps 0 and 1 apart (only lane 0
+  // runs the producer or issuer loop): reconverge each warp before the
+  // block-wide barrier, which counts whole warps.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
