@@ -212,20 +212,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     int cur = -1;
     float acc = 0.f;
     for (int c0 = 0; ok && c0 < nseg; c0 += 32) {
+      // the chunk's rows and weights, one segment per lane, handed round by
+      // shuffles (no shared-memory load between the stores below)
+      const int sl = c0 + lane;
+      const int row_l = sl < nseg ? sm.row[sl] : -1;
+      const float w_l = sl < nseg ? sm.w[sl] : 0.f;
       uint32_t d[32];
       tmem_ld32(tl + (uint32_t)c0, d);  // columns c0..c0+31 (the second MMA's start at 256)
       tmem_wait_ld();
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
-        const int s = c0 + k;
-        if (s >= nseg) break;
-        const int v = sm.row[s];
+        if (c0 + k >= nseg) break;  // the same for every lane
+        const int v = __shfl_sync(0xffffffffu, row_l, k);
+        const float w = __shfl_sync(0xffffffffu, w_l, k);
         if (v != cur) {
           if (cur >= 0) stage[cur * kVHead + f] = __float2bfloat16_rn(acc);
           cur = v;
           acc = 0.f;
         }
-        const float w = sm.w[s];
         if (w != 0.f) acc = fmaf(w, __uint_as_float(d[k]), acc);  // a zero weight: never-written partial
       }
     }
