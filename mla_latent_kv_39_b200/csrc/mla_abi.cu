@@ -288,11 +288,15 @@ mla_status absorb_tc(const mla_config* c, const void* x, int n, const void* W_DQ
   bf16* qn_lo = split ? reinterpret_cast<bf16*>(base + w.qn_lo) : nullptr;
   const ProjSpecs ps = proj_specs(c, n, split, W_DQ, W_UQ, W_UK, nullptr, nullptr, static_cast<const bf16*>(x),
                                   cq_hi, cq_lo, qn_hi, qn_lo, nullptr, nullptr);
+  // W_UQ head slice, RoPE and W_UK in one kernel; its rotation table (in the
+  // q_f region) depends on the positions only and is made first
+  const bool fused = qh::supports(c, n);
+  static_assert(sizeof(double) * 64 <= 4 * 192, "rotation table larger than the fp32 query it replaces");
+  if (fused) MLA_TRY(qh::launch_rope_table(c, n, pos, reinterpret_cast<double*>(q_f), s));
   if (c->q_lora > 0) MLA_TRY(wg::run(ps.dq, part, nullptr, cq_hi, cq_lo, s));
   const int H = c->n_heads, nope = c->qk_nope, row = c->d_c + c->d_r;
   bf16* qp_lo = q_packed && split ? q_packed + (long long)n * H * row : nullptr;
-  if (qh::supports(c, n)) {  // W_UQ head slice, RoPE and W_UK in one kernel (rotation table in the q_f region)
-    static_assert(sizeof(double) * 64 <= 4 * 192, "rotation table larger than the fp32 query it replaces");
+  if (fused) {
     return qh::launch(c, n, cq_hi, cq_lo, static_cast<const bf16*>(W_UQ), static_cast<const bf16*>(W_UK), pos,
                       reinterpret_cast<double*>(q_f), q_packed, qp_lo, q_packed ? nullptr : q_lat,
                       q_packed ? nullptr : q_rope, g_wait_limit_ns.load(std::memory_order_relaxed), s);

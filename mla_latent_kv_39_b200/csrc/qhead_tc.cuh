@@ -380,10 +380,21 @@ inline bool supports(const mla_config* c, int n_tok) {
 
 inline size_t rot_bytes(int n_tok) { return (size_t)n_tok * kRope * sizeof(double); }
 
+// The per-token rotation table `rot` (rot_bytes(n) bytes of device scratch)
+// that `launch` reads; it depends on the positions only, so it can be made
+// before the kernels that produce c_Q.
+inline mla_status launch_rope_table(const mla_config* c, int n, const int32_t* pos, double* rot, cudaStream_t s) {
+  const int pairs = n * (kRope / 2);
+  return launch_chained(rope_table_kernel, dim3((pairs + 255) / 256), dim3(256), 0, s, pos, n, c->rope_theta, rot) ==
+                 cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+
 // q_packed (bf16 [n][H][d_c + d_r], + remainders in split-query mode), or
 // with q_hi null the fp32 q_lat [n][H][d_c] and q_rope [n][H][d_r], from c_Q
 // (bf16 [n][q_lora], + remainders), W_UQ [q_lora, H (nope + d_r)] and W_UK
-// [d_c, H nope]; `rot` is a device scratch of rot_bytes(n) bytes.
+// [d_c, H nope]; `rot` holds the table of launch_rope_table, ordered before.
 inline mla_status launch(const mla_config* c, int n, const bf16* cq_hi, const bf16* cq_lo, const bf16* W_UQ,
                          const bf16* W_UK, const int32_t* pos, double* rot, bf16* q_hi, bf16* q_lo, float* q_lat,
                          float* q_rope, unsigned long long wait_ns, cudaStream_t s) {
@@ -451,10 +462,6 @@ inline mla_status launch(const mla_config* c, int n, const bf16* cq_hi, const bf
       if (bit) attr.fetch_or(bit, std::memory_order_acq_rel);
     }
   }
-  const int pairs = n * (kRope / 2);
-  if (launch_chained(rope_table_kernel, dim3((pairs + 255) / 256), dim3(256), 0, s, pos, n, c->rope_theta, rot) !=
-      cudaSuccess)
-    return MLA_ERR_CUDA;
   const Params p{n, H, c->q_lora / 64, rot, q_hi != nullptr ? 1 : 0, q_lat, q_rope, wait_ns};
   return launch_chained(kernel, dim3(H, (n + kTok - 1) / kTok), dim3(kThreads), kSmemBytes, s, uq, uk, cq, cql, ohi,
                         olo, p) == cudaSuccess

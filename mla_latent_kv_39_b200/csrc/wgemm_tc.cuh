@@ -130,26 +130,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  if (warp == 0 && lane == 0 && blockIdx.x < items) {
-    // The weights are not written by the kernels before this one: start
-    // pulling this CTA's first weight blocks into L2 while they finish.
-    int g, mt, kb0, kb1, s;
-    item_coords(p, blockIdx.x, g, mt, kb0, kb1, s);
-    for (int kb = kb0; kb < kb1 && kb < kb0 + nst; ++kb) {
-      if (p.a_kmajor) {
-        prefetch_l2_2d(&amap, g * p.a_g_stride + kb * 64, mt * 128);
-      } else {
-        prefetch_l2_2d(&amap, g * p.a_g_stride + mt * 128, kb * 64);
-        prefetch_l2_2d(&amap, g * p.a_g_stride + mt * 128 + 64, kb * 64);
-      }
-    }
+  if (warp != 0) {  // activations and output buffers belong to the kernels before
+    pdl_wait();
+    pdl_trigger();
   }
-  pdl_wait();  // activations and output buffers belong to the kernels before
-  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
+      auto load_a = [&](uint8_t* a, int g, int mt, int kb, uint64_t* bar) {
+        if (p.a_kmajor) {
+          tma_load_2d(a, &amap, g * p.a_g_stride + kb * 64, mt * 128, bar);
+        } else {
+          tma_load_2d(a, &amap, g * p.a_g_stride + mt * 128, kb * 64, bar);
+          tma_load_2d(a + kABytes / 2, &amap, g * p.a_g_stride + mt * 128 + 64, kb * 64, bar);
+        }
+      };
+      // The weights are not written by the kernels before this one: the first
+      // item's first stages of W go out before the wait, their activations after.
+      int pre = 0;
+      if (blockIdx.x < items) {
+        int g, mt, kb0, kb1, s;
+        item_coords(p, blockIdx.x, g, mt, kb0, kb1, s);
+        pre = min(nst, kb1 - kb0);
+        for (int i = 0; i < pre; ++i) {
+          mbar_arrive_expect_tx(&sm.full[i], stage_tx);
+          load_a(sm.ring + i * sbytes, g, mt, kb0 + i, &sm.full[i]);
+        }
+      }
+      pdl_wait();
+      pdl_trigger();
       int k = 0;
       for (int item = blockIdx.x; item < items && !aborted(sm); item += gridDim.x) {
         int g, mt, kb0, kb1, s;
@@ -162,18 +172,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* a = sm.ring + st * sbytes;
           uint8_t* b = a + kABytes;
-          mbar_arrive_expect_tx(&sm.full[st], stage_tx);
-          if (p.a_kmajor) {
-            tma_load_2d(a, &amap, g * p.a_g_stride + kb * 64, mt * 128, &sm.full[st]);
-          } else {
-            tma_load_2d(a, &amap, g * p.a_g_stride + mt * 128, kb * 64, &sm.full[st]);
-            tma_load_2d(a + kABytes / 2, &amap, g * p.a_g_stride + mt * 128 + 64, kb * 64, &sm.full[st]);
+          if (k >= pre) {
+            mbar_arrive_expect_tx(&sm.full[st], stage_tx);
+            load_a(a, g, mt, kb, &sm.full[st]);
           }
           tma_load_3d(b, &bmap_hi, kb * 64, g, 0, &sm.full[st]);
           if (p.split) tma_load_3d(b + b_bytes, &bmap_lo, kb * 64, g, 0, &sm.full[st]);
         }
       }
     producer_drain:
+      // no copy may be in flight when the CTA leaves (the weight stages issued
+      // before the wait included; a stage without its activations lands its
+      // weights long before this bounded wait gives up)
+      if (k < pre) k = pre;
       for (int kk = k - nst < 0 ? 0 : k - nst; kk < k; ++kk)
         mbar_wait(&sm.full[kk % nst], (kk / nst) & 1, 71);
     }
