@@ -173,3 +173,44 @@ def test_fused_projection_checks_its_arguments(lib):
     f32 = _cfg(dtype="f32")
     assert lib.mla_combine_out_proj_workspace_size(P(f32), 1, 1) == 0
 
+
+
+def test_fp8_cache_configuration_is_checked_before_any_launch(lib):
+    """MLA_FLAG_FP8_CACHE needs bf16 weights and the cache's row scales; the
+    packed-query (tensor-core) path does not take an FP8 cache."""
+    P = ctypes.byref
+    v3 = dict(hidden=7168, n_heads=128, d_c=512, d_r=64, qk_nope=128, v_head=128, q_lora=1536)
+    fp8 = abi.Config(**v3, dtype="bf16", fp8_cache=True).c()
+    assert fp8.flags & abi.MLA_FLAG_FP8_CACHE
+    f32 = _cfg(fp8_cache=True)                      # FP8 cache over fp32 weights: invalid
+    assert lib.mla_decode_workspace_size(P(f32), 1, 1, 0) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    no_scale = abi.MLACache(1 << 20, 4, 1 << 21, 1, 2, None)
+    need = lib.mla_decode_workspace_size(P(fp8), 1, 1, 8)
+    assert need > 0
+    assert lib.mla_decode(P(fp8), fake, fake, 1, 1, P(no_scale), fake, 8, fake, need, None) == abi.MLA_ERR_INVALID_ARG
+    assert lib.mla_cache_append(P(fp8), fake, 1, fake, fake, fake, fake, P(no_scale), fake, 1 << 30, None) \
+        == abi.MLA_ERR_INVALID_ARG
+    odd_scale = abi.MLACache(1 << 20, 4, 1 << 21, 1, 2, (1 << 22) + 2)   # not 4-byte aligned
+    assert lib.mla_decode(P(fp8), fake, fake, 1, 1, P(odd_scale), fake, 8, fake, need, None) == abi.MLA_ERR_INVALID_ARG
+    assert lib.mla_query_packed_bytes(P(fp8), 4) == 0
+    assert lib.mla_combine_out_proj_workspace_size(P(fp8), 64, 1) == 0
+    with_scale = abi.MLACache(1 << 20, 4, 1 << 21, 1, 2, 1 << 22)
+    assert lib.mla_decode_packed(P(fp8), fake, 1, 1, P(with_scale), fake, 8, fake, need, None) \
+        == abi.MLA_ERR_UNSUPPORTED
+    # the CUDA-core decode's workspace: fp32 partial outputs
+    bf = abi.Config(**v3, dtype="bf16").c()
+    assert lib.mla_decode_workspace_size(P(fp8), 64, 1, 74) > lib.mla_decode_workspace_size(P(bf), 64, 1, 74)
+
+
+def test_shard_merge_checks_its_arguments(lib):
+    P = ctypes.byref
+    c = _cfg()
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.mla_merge_shards(P(c), 0, 4, fake, fake, fake, None, None) == abi.MLA_ERR_INVALID_ARG
+    assert lib.mla_merge_shards(P(c), 2, -1, fake, fake, fake, None, None) == abi.MLA_ERR_INVALID_ARG
+    assert lib.mla_merge_shards(P(c), 2, 0, None, None, None, None, None) == abi.MLA_OK      # no rows
+    assert lib.mla_merge_shards(P(c), 2, 4, None, fake, fake, None, None) == abi.MLA_ERR_INVALID_ARG
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.mla_merge_shards(P(c), 2, 4, odd, fake, fake, None, None) == abi.MLA_ERR_INVALID_ARG
+    assert lib.mla_combine_lse(P(c), fake, 1 << 20, 1, 1, fake, None, None) == abi.MLA_ERR_INVALID_ARG
