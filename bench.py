@@ -116,7 +116,8 @@ def decode_roofline(wl, data, cache_bytes: int, dec_s: float, peaks, traffic):
     tensor_s = flops / (peaks["bf16_tflops"] * 1e12)
     kernel = "mla_decode_packed_planned call (the pair decode kernel; its split plan runs beside the query projections)"
     if wl.fp8_cache:
-        kernel = "mla_decode call (CUDA-core decode of the E4M3 cache rows and their scales, plan included)"
+        kernel = ("mla_cache_dequant_fp8 + mla_decode_packed_planned calls (the step's E4M3 pages expanded "
+                  "into a bf16 scratch cache, then the pair decode)")
     if wl.n_q > 1 and tensor_s > hbm_s:
         achieved = flops / dec_s / 1e12
         return {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",

@@ -102,9 +102,11 @@ typedef struct {
  * optimizasyonlarla ilişkisi": quantization is orthogonal to MLA and used
  * together with it; the pages fix no format, this is the plainest per-row
  * one).  A stored row [c_KV | k_R] stands for codes * scale with
- *   scale = fp32(max_i |row_i| / 448)   (1 when that is 0),
+ *   scale = the smallest power of two with max_i |row_i| / scale <= 448
+ *           (1 for a zero row), stored as fp32,
  *   code_i = E4M3(row_i / scale)        nearest, ties to even, from the exact
- *                                       fp64 row; saturating at +-448.
+ *                                       fp64 row.
+ * A power-of-two scale makes code * scale exact in bf16.
  * Requires dtype MLA_BF16 (weights and activations stay bf16) and
  * mla_cache.row_scale.  A 576-value row takes 580 bytes instead of 1152.
  * The decode of an FP8 cache runs on the CUDA-core path of mla_decode; the
@@ -233,6 +235,30 @@ mla_status mla_decode(const mla_config* cfg, const float* q_lat, const float* q_
                       int32_t batch, int32_t n_q, const mla_cache* cache,
                       const int32_t* seq_lens, int32_t max_workers,
                       void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * FP8 cache on the tensor-core decode (MLA_FLAG_FP8_CACHE; not on the pages):
+ * the visible pages of the step are expanded into a caller-owned bf16 scratch
+ * cache, which the bf16 entry points then decode (packed query, fused
+ * combine), with the configuration without MLA_FLAG_FP8_CACHE.
+ *   mla_fp8_scratch_bytes: bytes of that scratch for `batch` sequences of
+ *     up to `max_blocks_per_seq` pages (0 for a configuration without the
+ *     flag).  Layout: int32 block table [batch, max_blocks_per_seq], then,
+ *     256-byte aligned, bf16 pages [batch * max_blocks_per_seq, block_size,
+ *     d_c + d_r]; page (b, k) is scratch block b * max_blocks_per_seq + k.
+ *   mla_cache_dequant_fp8: for every sequence b < batch and page k holding
+ *     rows below seq_lens[b], scratch page (b, k) = bf16(code * row scale)
+ *     of cache page block_table[b][k]; writes the whole scratch block table.
+ *     Form the scratch cache as { pages, batch * max_blocks_per_seq, table,
+ *     batch, max_blocks_per_seq, NULL }.  The cache pool and the scratch must
+ *     be 16-byte aligned; d_c + d_r a multiple of 16.
+ * Errors: MLA_ERR_INVALID_ARG (flag missing, NULL or misaligned pointers, no
+ * row scales), MLA_ERR_WORKSPACE (scratch too small); bad lengths or block
+ * ids -> MLA_ERR_BOUNDS on the device error word (that page is not written).
+ * ------------------------------------------------------------------------- */
+size_t mla_fp8_scratch_bytes(const mla_config* cfg, int32_t batch, int32_t max_blocks_per_seq);
+mla_status mla_cache_dequant_fp8(const mla_config* cfg, const mla_cache* cache, int32_t batch,
+                                 const int32_t* seq_lens, void* scratch, size_t scratch_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Steps 2 and 3 with the query handed over in the decode's own layout

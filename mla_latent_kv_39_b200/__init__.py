@@ -19,6 +19,9 @@ from .abi import (  # noqa: F401
     mla_cache_append_noalloc,
     mla_combine,
     mla_combine_lse,
+    mla_cache_dequant_fp8,
+    mla_fp8_scratch_bytes,
+    fp8_scratch_cache,
     mla_combine_out_proj,
     mla_combine_out_proj_workspace_size,
     mla_decode,

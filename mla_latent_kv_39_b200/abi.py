@@ -65,6 +65,8 @@ SIGNATURES = {
     "mla_absorb_q_workspace_size": (_sz, [_P_CFG, _i32]),
     "mla_absorb_q": (_i32, [_P_CFG, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mla_query_packed_bytes": (_sz, [_P_CFG, _i32]),
+    "mla_fp8_scratch_bytes": (_sz, [_P_CFG, _i32, _i32]),
+    "mla_cache_dequant_fp8": (_i32, [_P_CFG, _P_CACHE, _i32, _vp, _vp, _sz, _vp]),
     "mla_absorb_q_packed": (_i32, [_P_CFG, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mla_decode_packed": (_i32, [_P_CFG, _vp, _i32, _i32, _P_CACHE, _vp, _i32, _vp, _sz, _vp]),
     "mla_decode_packed_planned": (_i32, [_P_CFG, _vp, _i32, _i32, _P_CACHE, _vp, _i32, _vp, _sz, _vp]),
@@ -352,6 +354,28 @@ def mla_combine(cfg: Config, workspace, batch: int, n_q: int, o_lat, stream=None
     _need(o_lat, "o_lat", torch.float32, shape=(batch * n_q, cfg.n_heads, cfg.d_c))
     _check(lib().mla_combine(ctypes.byref(cfg.c()), _ptr(workspace), workspace.numel(), batch, n_q,
                              _ptr(o_lat), _stream(stream)), "mla_combine")
+
+
+def mla_fp8_scratch_bytes(cfg: Config, batch: int, max_blocks_per_seq: int) -> int:
+    return int(lib().mla_fp8_scratch_bytes(ctypes.byref(cfg.c()), batch, max_blocks_per_seq))
+
+
+def fp8_scratch_cache(cfg: Config, scratch, batch: int, max_blocks_per_seq: int) -> "Cache":
+    """The bf16 cache view of an ``mla_cache_dequant_fp8`` scratch (layout in
+    ``include/mla.h``): decode it with ``cfg`` without ``fp8_cache``."""
+    _need(scratch, "scratch", torch.uint8)
+    slots = batch * max_blocks_per_seq
+    off = (4 * slots + 255) // 256 * 256
+    table = scratch[:4 * slots].view(torch.int32).view(batch, max_blocks_per_seq)
+    pages = scratch[off:off + slots * cfg.block_size * (cfg.d_c + cfg.d_r) * 2].view(torch.bfloat16)
+    return Cache(pages.view(slots, cfg.block_size, cfg.d_c + cfg.d_r), table)
+
+
+def mla_cache_dequant_fp8(cfg: Config, cache: "Cache", batch: int, seq_lens, scratch, stream=None):
+    _need(seq_lens, "seq_lens", torch.int32, shape=(batch,))
+    _need(scratch, "scratch", torch.uint8)
+    _check(lib().mla_cache_dequant_fp8(ctypes.byref(cfg.c()), ctypes.byref(cache.c), batch, _ptr(seq_lens),
+                                       _ptr(scratch), scratch.numel(), _stream(stream)), "mla_cache_dequant_fp8")
 
 
 def mla_combine_lse(cfg: Config, workspace, batch: int, n_q: int, o_lat, lse, stream=None):

@@ -89,8 +89,9 @@ __global__ void append_finish_kernel(const double* __restrict__ C, int splits, i
 
 // The same epilogue into an FP8 cache: one CTA per new token assembles its
 // exact row [c | RoPE(k_R)] in fp64 (shared memory), takes the row's largest
-// magnitude m, the scale s = fp32(m / 448) (1 if that is 0) and writes the
-// E4M3 codes of row / s (nearest, ties to even, saturating) and s.
+// magnitude m, the scale s = the smallest power of two with m / s <= 448 (1
+// if m is 0) and writes the E4M3 codes of row / s (nearest, ties to even)
+// and s.  A power-of-two scale keeps code * s exact in bf16.
 __global__ void __launch_bounds__(256) append_finish_fp8_kernel(
     const double* __restrict__ C, int n_tok, int d_c, int d_r, double theta, const int32_t* __restrict__ seq_idx,
     const int32_t* __restrict__ pos, __nv_fp8_e4m3* __restrict__ pool, float* __restrict__ row_scale,
@@ -126,11 +127,64 @@ __global__ void __launch_bounds__(256) append_finish_fp8_kernel(
   if (slot < 0) return;
   m = 0.0;
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmax(m, warp_max[w]);
-  float scale = __double2float_rn(m / 448.0);
+  // the smallest power of two s with m / s <= 448 (1 for a zero row)
+  int e = 0;
+  const double f = frexp(m / 448.0, &e);  // m / 448 = f 2^e, 0.5 <= f < 1
+  float scale = m > 0.0 ? (float)ldexp(1.0, f == 0.5 ? e - 1 : e) : 1.f;
   if (scale == 0.f) scale = 1.f;
   __nv_fp8_e4m3* dst = pool + slot * row;
   for (int k = threadIdx.x; k < row; k += blockDim.x) Store<__nv_fp8_e4m3>::st64(dst + k, v[k] / (double)scale);
   if (threadIdx.x == 0) row_scale[slot] = scale;
+}
+
+// FP8 cache pages -> bf16 pages for the tensor-core decode: page k of
+// sequence b (if visible) becomes scratch page b * max_blocks + k, each value
+// code * row scale rounded once to bf16, and the scratch block table entry
+// (b, k) = b * max_blocks + k.  Grid (max_blocks, batch); 16 codes per step.
+__global__ void __launch_bounds__(256) dequant_fp8_pages_kernel(
+    const uint8_t* __restrict__ pool, const float* __restrict__ row_scale, const int32_t* __restrict__ block_table,
+    int num_blocks, const int32_t* __restrict__ seq_lens, int max_blocks, int bs, int row,
+    bf16* __restrict__ out_pool, int32_t* __restrict__ out_table) {
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.y, k = blockIdx.x;
+  const long long slot = (long long)b * max_blocks + k;
+  if (threadIdx.x == 0) out_table[slot] = (int32_t)slot;
+  const int len = seq_lens[b];
+  if (len < 0 || len > max_blocks * bs) {
+    if (k == 0 && threadIdx.x == 0) report(MLA_ERR_BOUNDS, 6, b, len);
+    return;
+  }
+  const int rows = min(bs, len - k * bs);
+  if (rows <= 0) return;
+  const int phys = block_table[slot];
+  if (phys < 0 || phys >= num_blocks) {
+    if (threadIdx.x == 0) report(MLA_ERR_BOUNDS, 7, b, phys);
+    return;
+  }
+  const uint8_t* src = pool + (long long)phys * bs * row;
+  const float* sc = row_scale + (long long)phys * bs;
+  bf16* dst = out_pool + slot * bs * row;
+  const int per_row = row / 16;
+  for (int c = threadIdx.x; c < rows * per_row; c += blockDim.x) {
+    const float s = sc[c / per_row];
+    const uint4 in = *reinterpret_cast<const uint4*>(src + (long long)c * 16);
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t out[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      __nv_fp8_e4m3 lo, hi;
+      lo.__x = (__nv_fp8_storage_t)((w[i >> 1] >> (16 * (i & 1))) & 0xFFu);
+      hi.__x = (__nv_fp8_storage_t)((w[i >> 1] >> (16 * (i & 1) + 8)) & 0xFFu);
+      // code * scale is exact in fp64 (4 + 24 significant bits): one rounding to bf16
+      const bf16 a = __double2bfloat16((double)static_cast<float>(lo) * (double)s);
+      const bf16 c = __double2bfloat16((double)static_cast<float>(hi) * (double)s);
+      out[i] = (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(c) << 16);
+    }
+    uint4* o = reinterpret_cast<uint4*>(dst + (long long)c * 16);
+    o[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    o[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  }
 }
 
 // Split q [n, H, nope + d_r] (fp32) into q_nope (storage type) and the rotated

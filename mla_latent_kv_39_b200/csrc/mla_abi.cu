@@ -543,6 +543,33 @@ mla_status mla_absorb_q(const mla_config* cfg, const void* x, int32_t n_tok, con
   return absorb_impl<float>(cfg, x, n_tok, W_DQ, W_UQ, W_UK, pos, q_lat, q_rope, workspace, s);
 }
 
+size_t mla_fp8_scratch_bytes(const mla_config* cfg, int32_t batch, int32_t max_blocks_per_seq) {
+  if (check_cfg(cfg) != MLA_OK || !fp8_cache(cfg) || batch < 0 || max_blocks_per_seq <= 0) return 0;
+  const size_t slots = (size_t)batch * max_blocks_per_seq;
+  return align_up(4 * slots, 256) + slots * cfg->block_size * (cfg->d_c + cfg->d_r) * 2;
+}
+
+mla_status mla_cache_dequant_fp8(const mla_config* cfg, const mla_cache* cache, int32_t batch,
+                                 const int32_t* seq_lens, void* scratch, size_t scratch_bytes, void* stream) {
+  MLA_TRY(check_cfg(cfg));
+  if (!fp8_cache(cfg) || batch < 0) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!seq_lens || !scratch) return MLA_ERR_INVALID_ARG;
+  MLA_TRY(check_cache(cfg, cache));
+  if (cache->batch < batch) return MLA_ERR_INVALID_ARG;
+  const int row = cfg->d_c + cfg->d_r;
+  if (row % 16 != 0) return MLA_ERR_UNSUPPORTED;
+  if (!all_aligned16(cache->pool, scratch)) return MLA_ERR_INVALID_ARG;
+  if (scratch_bytes < mla_fp8_scratch_bytes(cfg, batch, cache->max_blocks_per_seq)) return MLA_ERR_WORKSPACE;
+  const size_t slots = (size_t)batch * cache->max_blocks_per_seq;
+  int32_t* table = static_cast<int32_t*>(scratch);
+  bf16* pages = reinterpret_cast<bf16*>(static_cast<char*>(scratch) + align_up(4 * slots, 256));
+  return st(launch_chained(dequant_fp8_pages_kernel, dim3(cache->max_blocks_per_seq, batch), dim3(256), 0,
+                           static_cast<cudaStream_t>(stream), static_cast<const uint8_t*>(cache->pool),
+                           (const float*)cache->row_scale, cache->block_table, cache->num_blocks, seq_lens,
+                           cache->max_blocks_per_seq, cfg->block_size, row, pages, table));
+}
+
 size_t mla_query_packed_bytes(const mla_config* cfg, int32_t n_tok) {
   if (check_cfg(cfg) != MLA_OK || n_tok < 0 || !tc_decode(cfg)) return 0;
   return (size_t)n_tok * pairdec::qpack_row_bytes(cfg);

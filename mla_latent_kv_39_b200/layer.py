@@ -25,6 +25,18 @@ class DecodeLayer:
         dev = cache.pool.device
         dt = cfg.torch_dtype
         H = cfg.n_heads
+        # An FP8 cache is appended as E4M3 rows; each step expands its visible
+        # pages into a bf16 scratch cache (mla_cache_dequant_fp8) that the bf16
+        # tensor-core path decodes: `dcfg` / `dcache` are what the queries, the
+        # decode and the projections see.
+        self.dcfg, self.dcache, self.fp8_scratch = cfg, cache, None
+        if cfg.fp8_cache and packed_query:
+            import dataclasses
+            self.dcfg = dataclasses.replace(cfg, fp8_cache=False)
+            mb = cache.block_table.shape[1]
+            self.fp8_scratch = torch.empty(abi.mla_fp8_scratch_bytes(cfg, batch, mb), dtype=torch.uint8, device=dev)
+            self.dcache = abi.fp8_scratch_cache(self.dcfg, self.fp8_scratch, batch, mb)
+        cfg = self.dcfg
         # bf16: the absorbed query goes from the projection to the decode in the
         # decode's packed bf16 layout (no fp32 round trip); fp32: q_lat / q_rope
         self.packed = packed_query and abi.mla_query_packed_bytes(cfg, n) > 0
@@ -66,10 +78,10 @@ class DecodeLayer:
         W_DQ = self.W.get("W_DQ")
         W_UQ = self.W["W_UQ"] if "W_UQ" in self.W else self.W["W_Q"]
         if self.packed:
-            abi.mla_absorb_q_packed(self.cfg, x, W_DQ, W_UQ, self.W["W_UK"], pos, self.q_packed, self.ws_gemm,
+            abi.mla_absorb_q_packed(self.dcfg, x, W_DQ, W_UQ, self.W["W_UK"], pos, self.q_packed, self.ws_gemm,
                                     stream)
         else:
-            abi.mla_absorb_q(self.cfg, x, W_DQ, W_UQ, self.W["W_UK"], pos, self.q_lat, self.q_rope,
+            abi.mla_absorb_q(self.dcfg, x, W_DQ, W_UQ, self.W["W_UK"], pos, self.q_lat, self.q_rope,
                              self.ws_gemm, stream)
 
     def queries_fp32(self):
@@ -80,9 +92,9 @@ class DecodeLayer:
             return self.q_lat, self.q_rope
         n = self.batch * self.n_q
         q = self.q_packed[:n].float()
-        if self.cfg.split_query:
+        if self.dcfg.split_query:
             q = q + self.q_packed[n:].float()
-        return q[..., :self.cfg.d_c], q[..., self.cfg.d_c:]
+        return q[..., :self.dcfg.d_c], q[..., self.dcfg.d_c:]
 
     def append_and_queries(self, x, seq_idx, pos, stream=None, seq_lens=None):
         """The append and the query projections of one step, overlapped: the
@@ -102,7 +114,7 @@ class DecodeLayer:
                              self.ws_append, self.side)
         keep = [x, seq_idx, pos]
         if seq_lens is not None and self.packed:
-            abi.mla_decode_plan(self.cfg, self.batch, self.n_q, self.cache, seq_lens, self.ws_decode,
+            abi.mla_decode_plan(self.dcfg, self.batch, self.n_q, self.dcache, seq_lens, self.ws_decode,
                                 self.max_workers, self.side)
             keep.append(seq_lens)
         done = torch.cuda.Event()
@@ -115,18 +127,20 @@ class DecodeLayer:
     def decode(self, seq_lens, stream=None, planned=False):
         """Split-KV decode; ``planned``: the plan is already in the workspace
         (``append_and_queries`` with ``seq_lens``, same sequence lengths)."""
+        if self.fp8_scratch is not None:   # this step's visible FP8 pages -> the bf16 scratch cache
+            abi.mla_cache_dequant_fp8(self.cfg, self.cache, self.batch, seq_lens, self.fp8_scratch, stream)
         if self.packed and planned:
-            abi.mla_decode_packed_planned(self.cfg, self.q_packed, self.batch, self.n_q, self.cache, seq_lens,
+            abi.mla_decode_packed_planned(self.dcfg, self.q_packed, self.batch, self.n_q, self.dcache, seq_lens,
                                           self.ws_decode, self.max_workers, stream)
         elif self.packed:
-            abi.mla_decode_packed(self.cfg, self.q_packed, self.batch, self.n_q, self.cache, seq_lens,
+            abi.mla_decode_packed(self.dcfg, self.q_packed, self.batch, self.n_q, self.dcache, seq_lens,
                                   self.ws_decode, self.max_workers, stream)
         else:
-            abi.mla_decode(self.cfg, self.q_lat, self.q_rope, self.batch, self.n_q, self.cache, seq_lens,
+            abi.mla_decode(self.dcfg, self.q_lat, self.q_rope, self.batch, self.n_q, self.dcache, seq_lens,
                            self.ws_decode, self.max_workers, stream)
 
     def combine(self, stream=None):
-        abi.mla_combine(self.cfg, self.ws_decode, self.batch, self.n_q, self.o_lat, stream)
+        abi.mla_combine(self.dcfg, self.ws_decode, self.batch, self.n_q, self.o_lat, stream)
 
     def attend(self, seq_lens, stream=None):
         """Decode, then the latent output ``o_lat`` (merged splits, fp32)."""
@@ -139,10 +153,10 @@ class DecodeLayer:
         ``o_lat`` (after ``combine``)."""
         y = self.y if y is None else y
         if self.fused_out:
-            abi.mla_combine_out_proj(self.cfg, self.ws_decode, self.batch, self.n_q, self.W["W_UV"], self.W["W_O"],
+            abi.mla_combine_out_proj(self.dcfg, self.ws_decode, self.batch, self.n_q, self.W["W_UV"], self.W["W_O"],
                                      y, self.ws_gemm, self.max_workers, stream)
         else:
-            abi.mla_out_proj(self.cfg, self.o_lat, self.W["W_UV"], self.W["W_O"], y, self.ws_gemm, stream)
+            abi.mla_out_proj(self.dcfg, self.o_lat, self.W["W_UV"], self.W["W_O"], y, self.ws_gemm, stream)
 
     def step(self, x, seq_idx, pos, seq_lens, stream=None, want_o_lat: bool = False) -> torch.Tensor:
         """Device-resident step: returns ``y`` ``[batch * n_q, hidden]`` (a reused buffer).

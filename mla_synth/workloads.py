@@ -20,10 +20,13 @@ with ``workload.seed`` (fixed so that every consumer sees identical values):
 5. the physical block permutation of the paged pool (``randperm``), when
    the workload asks for shuffled blocks;
 6. for an FP8 cache (``fp8_cache``), instead of step 4's latent rows: E4M3
-   codes ``[sum L_b, d_c + d_r]`` (sign, exponent field in 6..15 and
-   mantissa field uniform, never the NaN pattern: magnitudes 2^-1 .. 448)
-   and one fp32 scale per row, ``0.002 + 0.01 |N(0, 1)|``.  They are drawn
-   after step 5, as codes are stored bytes, not values.
+   codes ``[sum L_b, d_c + d_r]`` (sign uniform; exponent field 6..15 drawn
+   with the octave shares of a normal row whose 4-sigma value sits at 448;
+   mantissa field uniform; never the NaN pattern) and one scale per row, a
+   power of two as the format has it, ``2^k`` with k uniform in -8..-7
+   (rows of one layer have similar norms, so their maxima, and with them
+   the power-of-two scales, differ by about a factor of two).
+   They are drawn after step 5, as codes are stored bytes, not values.
 """
 
 from __future__ import annotations
@@ -253,6 +256,13 @@ def _draw_rows(n: int, width: int, dtype: torch.dtype, g: torch.Generator,
     return out
 
 
+# Share of the octaves [2^(e-7), 2^(e-6)) of |N(0, 1)| * 112 for exponent
+# fields e = 6 .. 15 (the lowest bin also takes everything below it, the top
+# one everything above 256): the magnitudes of a normal row whose 4-sigma
+# value is scaled to 448.
+_FP8_EXPONENT_WEIGHTS = (0.013, 0.007, 0.014, 0.028, 0.056, 0.11, 0.20, 0.32, 0.23, 0.022)
+
+
 def generate(wl: Workload, *, with_weights: bool = True) -> WorkloadData:
     """Draw every input of ``wl`` from its seed (see the module docstring)."""
     shape = wl.shape
@@ -311,11 +321,16 @@ def generate(wl: Workload, *, with_weights: bool = True) -> WorkloadData:
     codes = scales = None
     if wl.fp8_cache and not wl.cached_from_append:
         sign = torch.randint(0, 2, (total, shape.row), generator=g, dtype=torch.int32)
-        expo = torch.randint(6, 16, (total, shape.row), generator=g, dtype=torch.int32)
+        # exponent field 6..15 with the octave weights of |N(0, 1)| scaled so
+        # that 4 sigma lands on the largest code (a row quantised with its own
+        # max): most codes in [32, 256), a few percent at the top
+        octaves = torch.tensor(_FP8_EXPONENT_WEIGHTS, dtype=torch.float64)
+        expo = 6 + torch.multinomial(octaves, total * shape.row, replacement=True, generator=g)
+        expo = expo.view(total, shape.row).to(torch.int32)
         mant = torch.randint(0, 8, (total, shape.row), generator=g, dtype=torch.int32)
         mant = torch.where((expo == 15) & (mant == 7), torch.full_like(mant, 6), mant)   # 0x7F / 0xFF: NaN
         codes = ((sign << 7) | (expo << 3) | mant).to(torch.uint8)
-        scales = (0.002 + 0.01 * torch.randn(total, generator=g).abs()).to(torch.float32)
+        scales = torch.pow(2.0, torch.randint(-8, -6, (total,), generator=g).to(torch.float32))
 
     return WorkloadData(wl, weights, cached_len, x_new, cached_rows, x_cached, spike_mask,
                         block_table, num_blocks, row_offsets, codes, scales)

@@ -24,8 +24,9 @@ Parity status per function (pins live in ``tests/test_oracle_pins.py``):
                               float8_e4m3fn)
 * ``round_to_e4m3``           pinned (torch's fp32 -> float8_e4m3fn cast on fp32
                               values within +-448, ties, subnormals, saturation)
-* ``fp8_row_quantize``        pinned (the largest magnitude maps to 448, every value
-                              within half a code step, zero rows)
+* ``fp8_row_quantize``        pinned (power-of-two scales, the smallest that fit 448,
+                              the boundary case, every value within half a code step,
+                              zero rows, code x scale exact in bf16)
 """
 
 from .mla import (  # noqa: F401

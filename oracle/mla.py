@@ -127,14 +127,17 @@ def e4m3_code(values) -> np.ndarray:
 def fp8_row_quantize(rows) -> Tuple[np.ndarray, np.ndarray]:
     """Per-row scaled E4M3 of float64 rows ``[..., width]``.
 
-    ``scale = fp32(max |row| / 448)`` (1 where that is 0); the stored codes
-    are ``round_to_e4m3(row / scale)``.  Returns ``(code_values, scale)`` as
-    float64; the cached row stands for ``code_values * scale``.
+    ``scale`` = the smallest power of two with ``max |row| / scale <= 448``
+    (1 where the row is zero); the stored codes are ``round_to_e4m3(row /
+    scale)``.  Returns ``(code_values, scale)`` as float64; the cached row
+    stands for ``code_values * scale`` (exact in bf16: 4 significant bits
+    times a power of two).
     """
     r = np.asarray(rows, dtype=np.float64)
     amax = np.max(np.abs(r), axis=-1)
-    scale = (amax / _E4M3_MAX).astype(np.float32).astype(np.float64)
-    scale = np.where(scale == 0.0, 1.0, scale)
+    f, e = np.frexp(amax / _E4M3_MAX)          # amax / 448 = f 2**e, 0.5 <= f < 1
+    scale = np.ldexp(1.0, np.where(f == 0.5, e - 1, e))
+    scale = np.where(amax == 0.0, 1.0, scale)
     return round_to_e4m3(r / scale[..., None]), scale
 
 

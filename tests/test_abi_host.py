@@ -214,3 +214,21 @@ def test_shard_merge_checks_its_arguments(lib):
     odd = ctypes.c_void_p((1 << 20) + 8)
     assert lib.mla_merge_shards(P(c), 2, 4, odd, fake, fake, None, None) == abi.MLA_ERR_INVALID_ARG
     assert lib.mla_combine_lse(P(c), fake, 1 << 20, 1, 1, fake, None, None) == abi.MLA_ERR_INVALID_ARG
+
+
+def test_fp8_scratch_size_and_dequant_checks(lib):
+    P = ctypes.byref
+    v3 = dict(hidden=7168, n_heads=128, d_c=512, d_r=64, qk_nope=128, v_head=128, q_lora=1536)
+    fp8 = abi.Config(**v3, dtype="bf16", fp8_cache=True).c()
+    bf = abi.Config(**v3, dtype="bf16").c()
+    need = lib.mla_fp8_scratch_bytes(P(fp8), 3, 5)
+    assert need == 256 + 3 * 5 * 64 * 576 * 2          # table (60 B, padded to 256) + bf16 pages
+    assert lib.mla_fp8_scratch_bytes(P(bf), 3, 5) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    cache = abi.MLACache(1 << 20, 8, 1 << 21, 3, 5, 1 << 22)
+    assert lib.mla_cache_dequant_fp8(P(bf), P(cache), 3, fake, fake, need, None) == abi.MLA_ERR_INVALID_ARG
+    assert lib.mla_cache_dequant_fp8(P(fp8), P(cache), 3, fake, fake, need - 1, None) == abi.MLA_ERR_WORKSPACE
+    assert lib.mla_cache_dequant_fp8(P(fp8), P(cache), 3, None, fake, need, None) == abi.MLA_ERR_INVALID_ARG
+    assert lib.mla_cache_dequant_fp8(P(fp8), P(cache), 3, fake, ctypes.c_void_p((1 << 20) + 8), need, None) \
+        == abi.MLA_ERR_INVALID_ARG
+    assert lib.mla_cache_dequant_fp8(P(fp8), P(cache), 0, None, None, 0, None) == abi.MLA_OK

@@ -442,12 +442,23 @@ def test_round_to_e4m3_matches_torch_on_fp32_values_and_ties():
     assert np.signbit(oracle.round_to_e4m3(np.array([-2.0 ** -12]))[0])    # underflow keeps the sign
 
 
-def test_fp8_row_quantize_maps_the_row_maximum_to_448_within_half_a_step():
+def test_fp8_row_quantize_takes_the_smallest_power_of_two_scale_within_half_a_step():
     g = np.random.default_rng(9)
     rows = g.standard_normal((50, 576)) * np.exp(g.uniform(-8, 8, (50, 1)))
     codes, scale = oracle.fp8_row_quantize(rows)
-    assert np.all(scale == scale.astype(np.float32).astype(np.float64))       # fp32 scales
-    assert np.all(np.max(np.abs(codes), axis=1) == 448.0)
+    m, _ = np.frexp(scale)
+    assert np.all(m == 0.5)                                               # powers of two
+    amax = np.max(np.abs(rows), axis=1)
+    assert np.all(amax / scale <= 448.0) and np.all(amax / scale > 224.0)  # the smallest such power
+    big = np.max(np.abs(codes), axis=1)
+    assert np.all((big >= 224.0) & (big <= 448.0))       # (224, 448] rounds into [224, 448]
+    # a row whose max is exactly 448 * 2^k takes scale 2^k (the boundary case)
+    edge = np.zeros((1, 8))
+    edge[0, 3] = 448.0 * 2.0 ** -5
+    ce, se = oracle.fp8_row_quantize(edge)
+    assert se[0] == 2.0 ** -5 and ce[0, 3] == 448.0
+    # the stored value code * scale is a bf16 number (4 significant bits times 2^k)
+    assert np.array_equal(oracle.round_to_bf16(codes * scale[:, None]), codes * scale[:, None])
     # |row / s - code| <= half the code step at that magnitude (subnormal step 2^-9)
     _, e = np.frexp(np.abs(codes) + (codes == 0))
     step = np.ldexp(1.0, np.maximum(e - 4, -9))

@@ -68,3 +68,23 @@ def test_spiked_rows_are_scaled_by_eight():
     big = d.cached_rows[d.spike_mask].float().abs().mean()
     small = d.cached_rows[~d.spike_mask].float().abs().mean()
     assert 6.0 < float(big / small) < 10.0
+
+
+def test_fp8_workload_draws_codes_scales_and_keeps_the_weights():
+    from mla_synth import build_row_scale
+    wl = reduced(WORKLOADS["v3_fp8_b64_ragged1k_8k"], lengths=[70, 3])
+    data = generate(wl)
+    assert isinstance(data.weights, dict) and set(data.weights) >= {"W_DKV", "W_KR", "W_UK", "W_UV", "W_O"}
+    assert data.cached_rows is None and data.cached_codes.dtype == torch.uint8
+    assert data.cached_codes.shape == (73, wl.shape.row) and data.cached_scale.shape == (73,)
+    codes = data.cached_codes.to(torch.int64)
+    assert not bool(((codes & 0x7F) == 0x7F).any())            # never the NaN pattern
+    m, _ = torch.frexp(data.cached_scale)
+    assert bool((m == 0.5).all())                                   # powers of two, as the format has them
+    pool = build_pool(data)
+    scale = build_row_scale(data)
+    assert pool.dtype == torch.uint8 and scale.shape == pool.shape[:2]
+    b, t = 0, 65
+    phys = int(data.block_table[b, t // 64])
+    assert torch.equal(pool[phys, t % 64], data.cached_codes[t]) and scale[phys, t % 64] == data.cached_scale[t]
+    assert generate(wl).cached_codes.equal(data.cached_codes)    # seeded
