@@ -101,7 +101,10 @@ def decode_shard(cfg: abi.Config, q_packed: torch.Tensor, rows: int, cache: abi.
                  workspace: torch.Tensor, o_lat: torch.Tensor, lse: torch.Tensor, max_workers: int = 0,
                  stream=None) -> None:
     """This GPU's shard: every query row over the shard's rows (one query per
-    row), then its ``(o_lat, lse)``."""
+    row), then its ``(o_lat, lse)``.  The decode is the packed (tensor-core)
+    one: for an FP8 cache, expand the shard's pages first
+    (``mla_cache_dequant_fp8``) and pass the scratch cache with the
+    configuration without ``fp8_cache``."""
     abi.mla_decode_packed(cfg, q_packed, rows, 1, cache, seq_lens, workspace, max_workers, stream)
     abi.mla_combine_lse(cfg, workspace, rows, 1, o_lat, lse, stream)
 
