@@ -165,25 +165,38 @@ __global__ void __launch_bounds__(256) dequant_fp8_pages_kernel(
   const uint8_t* src = pool + (long long)phys * bs * row;
   const float* sc = row_scale + (long long)phys * bs;
   bf16* dst = out_pool + slot * bs * row;
-  const int per_row = row / 16;
-  for (int c = threadIdx.x; c < rows * per_row; c += blockDim.x) {
-    const float s = sc[c / per_row];
-    const uint4 in = *reinterpret_cast<const uint4*>(src + (long long)c * 16);
-    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-    uint32_t out[8];
+  const int per_row = row / 16, chunks = rows * per_row;
+  // kAhead 16-byte loads in flight per thread before any conversion
+  constexpr int kAhead = 4;
+  for (int c0 = threadIdx.x; c0 < chunks; c0 += kAhead * blockDim.x) {
+    uint4 buf[kAhead];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      __nv_fp8_e4m3 lo, hi;
-      lo.__x = (__nv_fp8_storage_t)((w[i >> 1] >> (16 * (i & 1))) & 0xFFu);
-      hi.__x = (__nv_fp8_storage_t)((w[i >> 1] >> (16 * (i & 1) + 8)) & 0xFFu);
-      // code * scale is exact in fp64 (4 + 24 significant bits): one rounding to bf16
-      const bf16 a = __double2bfloat16((double)static_cast<float>(lo) * (double)s);
-      const bf16 c = __double2bfloat16((double)static_cast<float>(hi) * (double)s);
-      out[i] = (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(c) << 16);
+    for (int j = 0; j < kAhead; ++j) {
+      const int c = c0 + j * blockDim.x;
+      if (c < chunks) buf[j] = __ldcs(reinterpret_cast<const uint4*>(src + (long long)c * 16));
     }
-    uint4* o = reinterpret_cast<uint4*>(dst + (long long)c * 16);
-    o[0] = make_uint4(out[0], out[1], out[2], out[3]);
-    o[1] = make_uint4(out[4], out[5], out[6], out[7]);
+#pragma unroll
+    for (int j = 0; j < kAhead; ++j) {
+      const int c = c0 + j * blockDim.x;
+      if (c >= chunks) break;
+      const float s = sc[c / per_row];
+      const uint4 in = buf[j];
+      const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+      uint32_t out[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        __nv_fp8_e4m3 lo, hi;
+        lo.__x = (__nv_fp8_storage_t)((w[i >> 1] >> (16 * (i & 1))) & 0xFFu);
+        hi.__x = (__nv_fp8_storage_t)((w[i >> 1] >> (16 * (i & 1) + 8)) & 0xFFu);
+        // code * scale is exact in fp64 (4 + 24 significant bits): one rounding to bf16
+        const bf16 va = __double2bfloat16((double)static_cast<float>(lo) * (double)s);
+        const bf16 vb = __double2bfloat16((double)static_cast<float>(hi) * (double)s);
+        out[i] = (uint32_t)__bfloat16_as_ushort(va) | ((uint32_t)__bfloat16_as_ushort(vb) << 16);
+      }
+      uint4* o = reinterpret_cast<uint4*>(dst + (long long)c * 16);
+      o[0] = make_uint4(out[0], out[1], out[2], out[3]);
+      o[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    }
   }
 }
 
