@@ -93,3 +93,38 @@ def test_gather_without_a_process_group_is_the_local_pair():
     o, lse = torch.ones(2, 3, 4), torch.zeros(2, 3)
     a, b = gather_partials(o, lse)
     assert a.shape == (1, 2, 3, 4) and b.shape == (1, 2, 3)
+
+
+def test_shard_plan_partials_merge_to_the_whole_attention():
+    """Host-side plan against the oracle: for every query row, attention over
+    each shard's visible rows (oracle), merged with the split merge, equals
+    attention over all the rows the row sees (empty shards left out, as their
+    lse is -inf on the device)."""
+    import numpy as np
+    import oracle
+    g = np.random.default_rng(3)
+    bs, H, d_c, d_r, n_q = 4, 2, 6, 2, 2
+    lens = torch.tensor([1 + n_q, 9, 23], dtype=torch.int32)          # pages: 1, 3, 6
+    batch = lens.numel()
+    mb = 6
+    bt = torch.arange(batch * mb, dtype=torch.int32).reshape(batch, mb)
+    rows = {b: g.standard_normal((int(lens[b]), d_c + d_r)) for b in range(batch)}
+    for n_shards in (2, 3, 4):
+        plan = shard_plan(bt, lens, n_q, bs, n_shards)
+        for b in range(batch):
+            for j in range(n_q):
+                v = b * n_q + j
+                q_lat, q_r = g.standard_normal((H, d_c)), g.standard_normal((H, d_r))
+                vis = int(lens[b]) - n_q + j + 1
+                whole, lse_whole, _ = oracle.attend_absorbed(q_lat, q_r, rows[b][:vis, :d_c], rows[b][:vis, d_c:], 0.3)
+                parts, lses = [], []
+                for r in range(n_shards):
+                    n = int(plan.seq_lens[r][v])
+                    if n == 0:
+                        continue
+                    lo = int(plan.page_bounds[b, r]) * bs
+                    o, lse, _ = oracle.attend_absorbed(q_lat, q_r, rows[b][lo:lo + n, :d_c], rows[b][lo:lo + n, d_c:], 0.3)
+                    parts.append(o)
+                    lses.append(lse)
+                o, lse = oracle.merge_splits(np.stack(parts), np.stack(lses))
+                assert np.allclose(o, whole, rtol=0, atol=1e-12) and np.allclose(lse, lse_whole, rtol=0, atol=1e-12)
