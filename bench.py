@@ -300,6 +300,53 @@ def run_reference(args):
     return 0
 
 
+def measure_sequence_split(layer, dev, wl, n_shards: int, steps: int, flush_l2):
+    """The sequence split across GPUs, its device work emulated on this GPU:
+    each shard's decode (its pages only, one query per row, then its
+    (o_lat, lse)) timed on its own, and the merge of the shards' pairs.  On
+    n_shards GPUs the shards run at once, so the split decode takes the
+    slowest shard plus the exchange (not run here: one GPU) plus the merge."""
+    import mla_latent_kv_39_b200 as mla
+    cfg, rows = layer.dcfg, wl.n_tok
+    if not layer.packed:
+        return {"shards": n_shards, "unavailable": "the sequence split decodes the packed bf16 query"}
+    plan = mla.shard_plan(dev["block_table"].cpu(), dev["seq_lens"].cpu(), wl.n_q, wl.shape.block_size, n_shards)
+    caches = [mla.Cache(dev["pool"], t.to(dev["pool"].device)) for t in plan.block_tables]
+    lens = [x.to(dev["pool"].device) for x in plan.seq_lens]
+    ws = torch.empty(mla.mla_decode_workspace_size(cfg, rows, 1, 0), dtype=torch.uint8, device=dev["pool"].device)
+    H, d_c = cfg.n_heads, cfg.d_c
+    o_parts = torch.empty(n_shards, rows, H, d_c, dtype=torch.float32, device=ws.device)
+    lse_parts = torch.empty(n_shards, rows, H, dtype=torch.float32, device=ws.device)
+    o = torch.empty(rows, H, d_c, dtype=torch.float32, device=ws.device)
+    shard_ms = [[] for _ in range(n_shards)]
+    merge_ms = []
+    for it in range(steps + 2):
+        for r in range(n_shards):
+            flush_l2()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            ev[0].record()
+            mla.decode_shard(cfg, layer.q_packed, rows, caches[r], lens[r], ws, o_parts[r], lse_parts[r])
+            ev[1].record()
+            torch.cuda.synchronize()
+            if it >= 2:
+                shard_ms[r].append(ev[0].elapsed_time(ev[1]))
+        flush_l2()   # also keeps the GPU busy while the host enqueues the timed launch
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record()
+        mla.mla_merge_shards(cfg, o_parts, lse_parts, o)
+        ev[1].record()
+        torch.cuda.synchronize()
+        if it >= 2:
+            merge_ms.append(ev[0].elapsed_time(ev[1]))
+    mla.check_device_error()
+    per_shard = [statistics.median(m) for m in shard_ms]
+    return {"shards": n_shards, "shard_decode_ms": per_shard, "slowest_shard_ms": max(per_shard),
+            "merge_ms": statistics.median(merge_ms),
+            "exchange_bytes_per_gpu": int(rows * H * (d_c + 1) * 4),
+            "note": "each shard's decode timed alone on one GPU (L2 flushed before); on one GPU per shard they "
+                    "run at once, plus an all-gather of the exchange bytes"}
+
+
 def run_ours(args):
     rank, world, local = dist_env()
     if not torch.cuda.is_available():
@@ -421,6 +468,10 @@ def run_ours(args):
     del graph
     mla.check_device_error()
 
+    split = None
+    if args.shards > 1 and world == 1:
+        split = measure_sequence_split(layer, dev, wl, args.shards, max(3, min(args.steps, 10)), flush_l2)
+
     peaks = measured_peaks()
     cache_bytes = int(data.seq_lens.sum()) * wl.cache_row_bytes
     dec_avg_s = statistics.mean(dec_ms) / 1000.0
@@ -468,6 +519,7 @@ def run_ours(args):
         "clocks": clocks.summary(),
         "wall_s_timed_region": wall,
         "cpu_baseline": cpu,
+        **({"sequence_split": split} if split is not None else {}),
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -483,6 +535,9 @@ def parse(argv=None):
     ap.add_argument("--max-workers", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shards", type=int, default=0,
+                    help="also time the sequence split across this many GPUs (emulated on one: each shard's "
+                         "decode alone, and the merge)")
     return ap.parse_args(argv)
 
 
