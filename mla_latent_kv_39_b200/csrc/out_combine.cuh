@@ -219,18 +219,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float w_l = sl < nseg ? sm.w[sl] : 0.f;
       uint32_t d[32];
       tmem_ld32(tl + (uint32_t)c0, d);  // columns c0..c0+31 (the second MMA's start at 256)
+      // every shuffle first (independent, pipelined), then a branch-free pass
+      int vk[32];
+      float wk[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        vk[k] = __shfl_sync(0xffffffffu, row_l, k);
+        wk[k] = __shfl_sync(0xffffffffu, w_l, k);
+      }
       tmem_wait_ld();
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
-        if (c0 + k >= nseg) break;  // the same for every lane
-        const int v = __shfl_sync(0xffffffffu, row_l, k);
-        const float w = __shfl_sync(0xffffffffu, w_l, k);
-        if (v != cur) {
-          if (cur >= 0) stage[cur * kVHead + f] = __float2bfloat16_rn(acc);
-          cur = v;
-          acc = 0.f;
-        }
-        if (w != 0.f) acc = fmaf(w, __uint_as_float(d[k]), acc);  // a zero weight: never-written partial
+        const int v = vk[k];       // -1 past the last segment: no row change, nothing to add
+        const bool next_row = v >= 0 && v != cur;
+        if (next_row && cur >= 0) stage[cur * kVHead + f] = __float2bfloat16_rn(acc);
+        acc = next_row ? 0.f : acc;
+        cur = next_row ? v : cur;
+        // a zero weight (also past the last segment): a never-written partial, skipped
+        acc = wk[k] != 0.f ? fmaf(wk[k], __uint_as_float(d[k]), acc) : acc;
       }
     }
     if (cur >= 0) stage[cur * kVHead + f] = __float2bfloat16_rn(acc);
