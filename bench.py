@@ -8,6 +8,12 @@ seed 0): the configuration on which the decode roofline target is stated.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the fp64 oracle on the host cores
+  python bench.py --workload v3_b4_long --shards 2   # also the sequence split
+
+Besides the eager step the line carries `e2e` (pinned host inputs and
+outputs through `DecodeLayer.run_from_host`), `graph_replay` (the step
+recorded once as a CUDA graph and replayed) and, with `--shards N`,
+`sequence_split` (each shard's decode and the merge, timed on one GPU).
 
 Timing: every step is bracketed by CUDA events on the stream the library
 launches on; the L2 is flushed before every step, outside the events (a
