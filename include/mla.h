@@ -33,8 +33,9 @@
  *    so stream order is kept exactly.
  *  - Ownership: the caller owns every buffer, including the workspaces whose
  *    sizes the *_workspace_size queries return.  The library allocates no
- *    device memory.  Its only device state is one error word per device
- *    (a file-scope __device__ variable).
+ *    device memory.  Its only device state, per device, is one error word
+ *    and the fixed scratch of mla_cache_append_noalloc (file-scope
+ *    __device__ variables).
  *  - Synchronous errors (null pointers, unsupported dimensions, workspace too
  *    small, a failed launch) return a negative mla_status before or at launch
  *    and leave outputs untouched.  Data-dependent errors found on the device
@@ -49,7 +50,8 @@
  *    pointer that does not returns MLA_ERR_INVALID_ARG.  mla_cache_append
  *    takes any alignment (unaligned operands take a slower kernel).
  *  - Storage dtype: MLA_BF16 (bf16 storage, fp32 accumulation) or MLA_F32
- *    (fp32 storage and arithmetic on CUDA cores, for small shapes).
+ *    (fp32 storage and arithmetic on CUDA cores, for small shapes); with
+ *    MLA_BF16 the cache alone may be FP8 (MLA_FLAG_FP8_CACHE).
  */
 #ifndef MLA_H_
 #define MLA_H_
